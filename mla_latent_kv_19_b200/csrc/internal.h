@@ -1,0 +1,101 @@
+// Internal declarations of libmla shared by the host C-ABI layer and the
+// kernel translation units.  Not part of the public interface (include/mla.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/mla.h"
+
+struct mla_ctx {
+  mla_config_t cfg;
+  int device;
+  int num_sms;
+  int cc_major, cc_minor;
+  float2* rope_cs;     // device [max_position][d_r/2] (cos, sin)
+  int* err;            // device error word (0 = no error)
+  uint32_t wait_limit; // bounded-wait iteration limit (0 = default)
+};
+
+namespace mla {
+
+constexpr uint32_t kDefaultWaitLimit = 1u << 26;
+
+// Counts kernel launches (host side); read through mla_launch_count().
+void note_launches(int n);
+
+// Work description shared by the append kernels.
+struct AppendArgs {
+  const void* c_kv;     // [T, d_c]   (append)
+  const void* k_r;      // [T, d_r]   (append)
+  const void* x;        // [T, d_model] (project-append)
+  const void* w_dkv;    // [d_c, d_model]
+  const void* w_kr;     // [d_r, d_model]
+  const int32_t* seq_idx;
+  const int32_t* pos;
+  int32_t num_tokens;
+  const int32_t* block_table;
+  int32_t max_blocks;
+  int32_t batch;
+  void* cache;
+  float* cache_scale;
+  int32_t num_blocks;
+  const float2* rope_cs;
+  int* err;
+  int32_t d_c, d_r, d_model, block_size, max_position;
+};
+
+struct AbsorbArgs {
+  const void* q_nope;   // [B, H, d_nope]
+  const void* q_pe;     // [B, H, d_r]
+  const int32_t* pos;   // [B]
+  const void* w_uk;     // [H, d_nope, d_c]
+  void* q_lat;          // [B, H, d_c + d_r]
+  const float2* rope_cs;
+  int* err;
+  int32_t batch, num_heads, d_nope, d_c, d_r, max_position;
+};
+
+struct DecodeArgs {
+  const void* q_lat;          // [B, H, D]
+  const void* cache;          // [num_blocks, block_size, D]
+  const float* cache_scale;   // [num_blocks, block_size] (fp8)
+  const int32_t* block_table; // [B, max_blocks]
+  const int32_t* seq_lens;    // [B]
+  float* o_part;              // [B, S, H, d_c]
+  float* lse_part;            // [B, S, H]
+  int* err;
+  int32_t batch, num_heads, d_c, d_r, block_size, max_blocks, num_splits, num_blocks;
+  int32_t max_seq_len;
+  float scale;
+  uint32_t wait_limit;
+};
+
+struct CombineArgs {
+  const float* o_part;
+  const float* lse_part;
+  void* o_lat;                // [B, H, d_c] act dtype
+  float* lse;                 // [B, H] or null
+  int32_t batch, num_heads, d_c, num_splits;
+};
+
+struct OutProjArgs {
+  const void* o_lat;   // [B, H, d_c]
+  const void* w_uv;    // [H, d_v, d_c]
+  const void* w_o;     // [d_model, H*d_v]
+  void* o;             // [B, H, d_v]
+  void* y;             // [B, d_model]
+  int32_t batch, num_heads, d_c, d_v, d_model;
+};
+
+// Launchers (return cudaGetLastError() of their launches).
+cudaError_t launch_append(const AppendArgs& a, int act_dtype, int cache_dtype, bool project,
+                          cudaStream_t s);
+cudaError_t launch_absorb_generic(const AbsorbArgs& a, int act_dtype, cudaStream_t s);
+cudaError_t launch_decode_generic(const DecodeArgs& a, int act_dtype, int cache_dtype,
+                                  cudaStream_t s);
+cudaError_t launch_combine(const CombineArgs& a, int act_dtype, cudaStream_t s);
+cudaError_t launch_out_proj_generic(const OutProjArgs& a, int act_dtype, cudaStream_t s);
+
+}  // namespace mla

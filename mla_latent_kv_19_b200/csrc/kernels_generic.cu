@@ -1,0 +1,566 @@
+// CUDA-core kernels of libmla that serve every configuration:
+//   * the paged row write (append and project-append), the split merge and
+//     the RoPE of the query -- element-wise, HBM/latency bound at every size;
+//   * dimension-generic absorb / decode / output projections, used for shapes
+//     the tensor-core kernels are not specialised for (e.g. the tiny fp32
+//     configuration with H=8, d_c=64, d_r=16).
+//
+// Method: DeepSeek V2 MLA page (snabindia.com), sections 2.1-2.3.
+#include "device_common.cuh"
+
+namespace mla {
+
+// ---------------------------------------------------------------------------
+// paged row write (V2 page section 2.2 mla_rope, section 2.3 cache layout)
+// ---------------------------------------------------------------------------
+
+constexpr int kAppendWarps = 4;
+
+// Writes one token's row from a staged fp32 copy (c_KV then raw k_R) held in
+// shared memory by one warp.  RoPE pairs (i, i + d_r/2).
+template <typename CT>
+__device__ void write_row_warp(const AppendArgs& a, const float* stage, int p, long slot,
+                               int lane) {
+  const int D = a.d_c + a.d_r;
+  const int half = a.d_r / 2;
+  const float2* cs = a.rope_cs + static_cast<long>(p) * half;
+  CT* row = reinterpret_cast<CT*>(a.cache) + slot * D;
+  for (int i = lane; i < a.d_c; i += 32) row[i] = cvt_out<CT>(stage[i]);
+  for (int i = lane; i < half; i += 32) {
+    const float x1 = stage[a.d_c + i], x2 = stage[a.d_c + half + i];
+    const float2 r = cs[i];
+    row[a.d_c + i] = cvt_out<CT>(x1 * r.x - x2 * r.y);
+    row[a.d_c + half + i] = cvt_out<CT>(x2 * r.x + x1 * r.y);
+  }
+}
+
+__device__ void write_row_warp_fp8(const AppendArgs& a, float* stage, int p, long slot, int lane) {
+  const int D = a.d_c + a.d_r;
+  const int half = a.d_r / 2;
+  const float2* cs = a.rope_cs + static_cast<long>(p) * half;
+  // rotate k in place (each pair is owned by one lane)
+  for (int i = lane; i < half; i += 32) {
+    const float x1 = stage[a.d_c + i], x2 = stage[a.d_c + half + i];
+    const float2 r = cs[i];
+    stage[a.d_c + i] = x1 * r.x - x2 * r.y;
+    stage[a.d_c + half + i] = x2 * r.x + x1 * r.y;
+  }
+  __syncwarp();
+  float amax = 0.f;
+  for (int i = lane; i < D; i += 32) amax = fmaxf(amax, fabsf(stage[i]));
+  amax = warp_max(amax);
+  uint8_t* row = reinterpret_cast<uint8_t*>(a.cache) + slot * D;
+  if (amax == 0.f) {
+    for (int i = lane; i < D; i += 32) row[i] = 0;
+    if (lane == 0) a.cache_scale[slot] = 1.f;
+    return;
+  }
+  const float inv = 448.f / amax;
+  for (int i = lane; i < D; i += 32) row[i] = encode_e4m3(stage[i] * inv);
+  if (lane == 0) a.cache_scale[slot] = amax / 448.f;
+}
+
+// Resolve the physical slot of token t; false (and an error report) if the
+// sequence, position or page is out of range.
+__device__ __forceinline__ bool resolve_slot(const AppendArgs& a, int t, int* p_out, long* slot) {
+  const int b = a.seq_idx ? a.seq_idx[t] : t;
+  const int p = a.pos[t];
+  if (b < 0 || b >= a.batch || p < 0 || p >= a.max_position ||
+      p / a.block_size >= a.max_blocks) {
+    return false;
+  }
+  const int page = a.block_table[static_cast<long>(b) * a.max_blocks + p / a.block_size];
+  if (page < 0 || page >= a.num_blocks) return false;
+  *p_out = p;
+  *slot = static_cast<long>(page) * a.block_size + p % a.block_size;
+  return true;
+}
+
+template <typename T, typename CT, bool kFp8, bool kProject>
+__global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(AppendArgs a) {
+  extern __shared__ float smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int D = a.d_c + a.d_r;
+  const int t = blockIdx.x * kAppendWarps + warp;
+  if (t >= a.num_tokens) return;
+  int p;
+  long slot;
+  if (!resolve_slot(a, t, &p, &slot)) {
+    if (lane == 0) report_error(a.err, MLA_ERR_BAD_INDEX);
+    return;
+  }
+  float* stage = smem + warp * D;
+  if (kProject) {
+    // c_kv = W_DKV x, k_raw = W_KR x: one output per warp iteration, lanes over d_model
+    float* xs = smem + kAppendWarps * D + warp * a.d_model;
+    const T* x = reinterpret_cast<const T*>(a.x) + static_cast<long>(t) * a.d_model;
+    for (int i = lane; i < a.d_model; i += 32) xs[i] = ld_f32(x, i);
+    __syncwarp();
+    for (int j = 0; j < D; ++j) {
+      const T* w = j < a.d_c ? reinterpret_cast<const T*>(a.w_dkv) + static_cast<long>(j) * a.d_model
+                             : reinterpret_cast<const T*>(a.w_kr) +
+                                   static_cast<long>(j - a.d_c) * a.d_model;
+      float acc = 0.f;
+      for (int i = lane; i < a.d_model; i += 32) acc += ld_f32(w, i) * xs[i];
+      acc = warp_sum(acc);
+      if (lane == 0) stage[j] = acc;
+    }
+  } else {
+    const T* c = reinterpret_cast<const T*>(a.c_kv) + static_cast<long>(t) * a.d_c;
+    const T* k = reinterpret_cast<const T*>(a.k_r) + static_cast<long>(t) * a.d_r;
+    for (int i = lane; i < a.d_c; i += 32) stage[i] = ld_f32(c, i);
+    for (int i = lane; i < a.d_r; i += 32) stage[a.d_c + i] = ld_f32(k, i);
+  }
+  __syncwarp();
+  if constexpr (kFp8) {
+    write_row_warp_fp8(a, stage, p, slot, lane);
+  } else {
+    write_row_warp<CT>(a, stage, p, slot, lane);
+  }
+}
+
+cudaError_t launch_append(const AppendArgs& a, int act_dtype, int cache_dtype, bool project,
+                          cudaStream_t s) {
+  if (a.num_tokens == 0) return cudaSuccess;
+  const int D = a.d_c + a.d_r;
+  size_t smem = sizeof(float) * kAppendWarps * (D + (project ? a.d_model : 0));
+  dim3 grid((a.num_tokens + kAppendWarps - 1) / kAppendWarps), block(kAppendWarps * 32);
+  void (*k)(AppendArgs) = nullptr;
+  if (act_dtype == MLA_FP32 && cache_dtype == MLA_FP32) {
+    k = project ? append_kernel<float, float, false, true> : append_kernel<float, float, false, false>;
+  } else if (act_dtype == MLA_BF16 && cache_dtype == MLA_BF16) {
+    k = project ? append_kernel<__nv_bfloat16, __nv_bfloat16, false, true>
+                : append_kernel<__nv_bfloat16, __nv_bfloat16, false, false>;
+  } else if (act_dtype == MLA_BF16 && cache_dtype == MLA_FP8_E4M3) {
+    k = project ? append_kernel<__nv_bfloat16, uint8_t, true, true>
+                : append_kernel<__nv_bfloat16, uint8_t, true, false>;
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  k<<<grid, block, smem, s>>>(a);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// absorbed query, dimension-generic (V2 page section 2.3)
+// ---------------------------------------------------------------------------
+
+constexpr int kAbsorbThreads = 128;
+constexpr int kAbsorbBatchChunk = 32;
+
+// grid (H, ceil(d_c / 128) + 1): the last y-slice applies RoPE to q_pe.
+template <typename T>
+__global__ void __launch_bounds__(kAbsorbThreads) absorb_generic_kernel(AbsorbArgs a) {
+  extern __shared__ float qs[];  // [kAbsorbBatchChunk][d_nope]
+  const int h = blockIdx.x;
+  const int D = a.d_c + a.d_r;
+  const int nslices = (a.d_c + kAbsorbThreads - 1) / kAbsorbThreads;
+  T* out = reinterpret_cast<T*>(a.q_lat);
+  if (static_cast<int>(blockIdx.y) == nslices) {
+    const int half = a.d_r / 2;
+    const T* qpe = reinterpret_cast<const T*>(a.q_pe);
+    for (int idx = threadIdx.x; idx < a.batch * half; idx += blockDim.x) {
+      const int b = idx / half, i = idx % half;
+      const int p = a.pos[b];
+      if (p < 0 || p >= a.max_position) {
+        report_error(a.err, MLA_ERR_BAD_INDEX);
+        continue;
+      }
+      const float2 r = a.rope_cs[static_cast<long>(p) * half + i];
+      const long base = (static_cast<long>(b) * a.num_heads + h) * a.d_r;
+      const float x1 = ld_f32(qpe, base + i), x2 = ld_f32(qpe, base + half + i);
+      const long ob = (static_cast<long>(b) * a.num_heads + h) * D + a.d_c;
+      out[ob + i] = cvt_out<T>(x1 * r.x - x2 * r.y);
+      out[ob + half + i] = cvt_out<T>(x2 * r.x + x1 * r.y);
+    }
+    return;
+  }
+  const int c = blockIdx.y * kAbsorbThreads + threadIdx.x;
+  const T* qn = reinterpret_cast<const T*>(a.q_nope);
+  const T* w = reinterpret_cast<const T*>(a.w_uk) + static_cast<long>(h) * a.d_nope * a.d_c;
+  for (int b0 = 0; b0 < a.batch; b0 += kAbsorbBatchChunk) {
+    const int nb = min(kAbsorbBatchChunk, a.batch - b0);
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < nb * a.d_nope; idx += blockDim.x) {
+      const int i = idx / a.d_nope, k = idx % a.d_nope;
+      qs[i * a.d_nope + k] = ld_f32(qn, (static_cast<long>(b0 + i) * a.num_heads + h) * a.d_nope + k);
+    }
+    __syncthreads();
+    if (c < a.d_c) {
+      float acc[kAbsorbBatchChunk];
+#pragma unroll
+      for (int i = 0; i < kAbsorbBatchChunk; ++i) acc[i] = 0.f;
+      for (int k = 0; k < a.d_nope; ++k) {
+        const float wv = ld_f32(w, static_cast<long>(k) * a.d_c + c);
+#pragma unroll
+        for (int i = 0; i < kAbsorbBatchChunk; ++i) acc[i] += wv * qs[i * a.d_nope + k];
+      }
+      for (int i = 0; i < nb; ++i)
+        out[(static_cast<long>(b0 + i) * a.num_heads + h) * D + c] = cvt_out<T>(acc[i]);
+    }
+  }
+}
+
+cudaError_t launch_absorb_generic(const AbsorbArgs& a, int act_dtype, cudaStream_t s) {
+  if (a.batch == 0) return cudaSuccess;
+  dim3 grid(a.num_heads, (a.d_c + kAbsorbThreads - 1) / kAbsorbThreads + 1);
+  size_t smem = sizeof(float) * kAbsorbBatchChunk * a.d_nope;
+  if (act_dtype == MLA_FP32) {
+    absorb_generic_kernel<float><<<grid, kAbsorbThreads, smem, s>>>(a);
+  } else {
+    absorb_generic_kernel<__nv_bfloat16><<<grid, kAbsorbThreads, smem, s>>>(a);
+  }
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// split-KV decode, dimension-generic (CUDA cores)
+// ---------------------------------------------------------------------------
+// One CTA per (sequence b, split s, group of up to 16 heads).  Tiles of 32
+// tokens are staged in shared memory as fp32 (fp8 rows are dequantised with
+// their per-token scale); every warp owns two heads and runs the online
+// softmax over the tile's 32 scores with warp-shuffle reductions.
+
+constexpr int kGenThreads = 256;
+constexpr int kGenTile = 32;
+constexpr int kGenHeads = 16;
+constexpr int kGenColsPerThread = 2;   // d_c <= 512
+
+template <typename T, typename CT, bool kFp8>
+__global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(DecodeArgs a) {
+  extern __shared__ float sm[];
+  const int D = a.d_c + a.d_r;
+  const int b = blockIdx.x, split = blockIdx.y, hg = blockIdx.z;
+  const int h0 = hg * kGenHeads;
+  const int nh = min(kGenHeads, a.num_heads - h0);
+  float* qs = sm;                           // [kGenHeads][D]
+  float* ks = qs + kGenHeads * D;           // [kGenTile][D]
+  float* ps = ks + kGenTile * D;            // [kGenHeads][kGenTile]
+  float* alpha_s = ps + kGenHeads * kGenTile;  // [kGenHeads]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  int len = a.seq_lens[b];
+  const int cap = a.max_blocks * a.block_size;
+  if (len < 0 || len > cap) {          // never read past the page-table row
+    if (tid == 0) report_error(a.err, MLA_ERR_BAD_INDEX);
+    len = len < 0 ? 0 : cap;
+  }
+  // token range of this split: pages divided evenly over the splits
+  const int pages = (len + a.block_size - 1) / a.block_size;
+  const int pps = (pages + a.num_splits - 1) / a.num_splits;
+  const int t_begin = min(len, split * pps * a.block_size);
+  const int t_end = min(len, (split + 1) * pps * a.block_size);
+
+  const T* q = reinterpret_cast<const T*>(a.q_lat);
+  for (int idx = tid; idx < kGenHeads * D; idx += kGenThreads) {
+    const int g = idx / D, d = idx % D;
+    qs[idx] = g < nh ? ld_f32(q, (static_cast<long>(b) * a.num_heads + h0 + g) * D + d) : 0.f;
+  }
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};   // heads 2*warp, 2*warp+1
+  float acc[kGenHeads][kGenColsPerThread];
+#pragma unroll
+  for (int g = 0; g < kGenHeads; ++g)
+#pragma unroll
+    for (int j = 0; j < kGenColsPerThread; ++j) acc[g][j] = 0.f;
+
+  const float sl2 = a.scale * 1.4426950408889634f;   // scores in log2 units
+  for (int t0 = t_begin; t0 < t_end; t0 += kGenTile) {
+    const int nt = min(kGenTile, t_end - t0);
+    __syncthreads();
+    // stage the tile
+    for (int idx = tid; idx < kGenTile * D; idx += kGenThreads) {
+      const int j = idx / D, d = idx % D;
+      float v = 0.f;
+      if (j < nt) {
+        const int tok = t0 + j;
+        const int page = a.block_table[static_cast<long>(b) * a.max_blocks + tok / a.block_size];
+        if (page >= 0 && page < a.num_blocks) {
+          const long slot = static_cast<long>(page) * a.block_size + tok % a.block_size;
+          if constexpr (kFp8) {
+            v = decode_e4m3(reinterpret_cast<const uint8_t*>(a.cache)[slot * D + d]) *
+                a.cache_scale[slot];
+          } else {
+            v = ld_f32(reinterpret_cast<const CT*>(a.cache), slot * D + d);
+          }
+        } else if (d == 0) {
+          report_error(a.err, MLA_ERR_BAD_INDEX);
+        }
+      }
+      ks[idx] = v;
+    }
+    __syncthreads();
+    // scores: warp w handles heads 2w, 2w+1; lane j handles token j
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int g = warp * 2 + hh;
+      float s = -INFINITY;
+      if (g < nh && lane < nt) {
+        float dot = 0.f;
+        const float* qg = qs + g * D;
+        const float* kj = ks + lane * D;
+        // lanes start at different columns so the 32 rows hit 32 banks
+        for (int dd = 0; dd < D; ++dd) {
+          int d = dd + lane;
+          if (d >= D) d -= D;
+          dot += qg[d] * kj[d];
+        }
+        s = dot * sl2;
+      }
+      const float m_tile = warp_max(s);
+      const float m_new = fmaxf(m_run[hh], m_tile);
+      const float p = (g < nh && lane < nt) ? exp2f(s - m_new) : 0.f;
+      const float alpha = (m_run[hh] == -INFINITY) ? 0.f : exp2f(m_run[hh] - m_new);
+      l_run[hh] = l_run[hh] * alpha + warp_sum(p);
+      m_run[hh] = m_new;
+      if (g < kGenHeads) {
+        ps[g * kGenTile + lane] = p;
+        if (lane == 0) alpha_s[g] = alpha;
+      }
+    }
+    __syncthreads();
+    // O[g][c] = alpha_g O[g][c] + sum_j p[g][j] row_j[c]
+#pragma unroll
+    for (int jc = 0; jc < kGenColsPerThread; ++jc) {
+      const int c = tid + jc * kGenThreads;
+      if (c < a.d_c) {
+#pragma unroll
+        for (int g = 0; g < kGenHeads; ++g) {
+          float o = acc[g][jc] * alpha_s[g];
+          for (int j = 0; j < nt; ++j) o += ps[g * kGenTile + j] * ks[j * D + c];
+          acc[g][jc] = o;
+        }
+      }
+    }
+  }
+  // write the normalised partial and its log-sum-exp
+  __syncthreads();
+  if (lane == 0) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int g = warp * 2 + hh;
+      if (g < kGenHeads) {
+        ps[g] = l_run[hh];                       // reuse: l per head
+        alpha_s[g] = m_run[hh];                  // reuse: m per head (log2 units)
+      }
+    }
+  }
+  __syncthreads();
+  const long part = (static_cast<long>(b) * a.num_splits + split) * a.num_heads;
+#pragma unroll
+  for (int jc = 0; jc < kGenColsPerThread; ++jc) {
+    const int c = tid + jc * kGenThreads;
+    if (c < a.d_c) {
+#pragma unroll
+      for (int g = 0; g < kGenHeads; ++g) {
+        if (g < nh) {
+          const float l = ps[g];
+          a.o_part[(part + h0 + g) * a.d_c + c] = l > 0.f ? acc[g][jc] / l : 0.f;
+        }
+      }
+    }
+  }
+  if (tid < nh) {
+    const float l = ps[tid];
+    a.lse_part[part + h0 + tid] =
+        l > 0.f ? (alpha_s[tid] + log2f(l)) * 0.6931471805599453f : -INFINITY;
+  }
+}
+
+cudaError_t launch_decode_generic(const DecodeArgs& a, int act_dtype, int cache_dtype,
+                                  cudaStream_t s) {
+  if (a.batch == 0) return cudaSuccess;
+  if (a.d_c > kGenThreads * kGenColsPerThread) return cudaErrorInvalidValue;
+  const int D = a.d_c + a.d_r;
+  dim3 grid(a.batch, a.num_splits, (a.num_heads + kGenHeads - 1) / kGenHeads);
+  size_t smem = sizeof(float) * (kGenHeads * D + kGenTile * D + kGenHeads * kGenTile + kGenHeads);
+  void (*k)(DecodeArgs) = nullptr;
+  if (act_dtype == MLA_FP32 && cache_dtype == MLA_FP32) {
+    k = decode_generic_kernel<float, float, false>;
+  } else if (act_dtype == MLA_BF16 && cache_dtype == MLA_BF16) {
+    k = decode_generic_kernel<__nv_bfloat16, __nv_bfloat16, false>;
+  } else if (act_dtype == MLA_BF16 && cache_dtype == MLA_FP8_E4M3) {
+    k = decode_generic_kernel<__nv_bfloat16, uint8_t, true>;
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  k<<<grid, kGenThreads, smem, s>>>(a);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// split merge by log-sum-exp
+// ---------------------------------------------------------------------------
+
+template <typename T>
+__global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
+  extern __shared__ float w_s[];  // [num_splits]
+  __shared__ float inv_z_s, lse_s;
+  const int b = blockIdx.x, h = blockIdx.y;
+  const int S = a.num_splits;
+  const long part0 = static_cast<long>(b) * S * a.num_heads + h;
+  if (threadIdx.x < 32) {
+    float m = -INFINITY;
+    for (int s = threadIdx.x; s < S; s += 32) m = fmaxf(m, a.lse_part[part0 + static_cast<long>(s) * a.num_heads]);
+    m = warp_max(m);
+    float z = 0.f;
+    for (int s = threadIdx.x; s < S; s += 32) {
+      const float l = a.lse_part[part0 + static_cast<long>(s) * a.num_heads];
+      const float w = (m == -INFINITY) ? 0.f : __expf(l - m);
+      w_s[s] = w;
+      z += w;
+    }
+    z = warp_sum(z);
+    if (threadIdx.x == 0) {
+      inv_z_s = z > 0.f ? 1.f / z : 0.f;
+      lse_s = z > 0.f ? m + __logf(z) : -INFINITY;
+    }
+  }
+  __syncthreads();
+  const float inv_z = inv_z_s;
+  T* out = reinterpret_cast<T*>(a.o_lat) + (static_cast<long>(b) * a.num_heads + h) * a.d_c;
+  for (int c = threadIdx.x; c < a.d_c; c += blockDim.x) {
+    float o = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float w = w_s[s];
+      if (w != 0.f) o += w * a.o_part[(part0 + static_cast<long>(s) * a.num_heads) * a.d_c + c];
+    }
+    out[c] = cvt_out<T>(o * inv_z);
+  }
+  if (threadIdx.x == 0 && a.lse != nullptr) a.lse[static_cast<long>(b) * a.num_heads + h] = lse_s;
+}
+
+cudaError_t launch_combine(const CombineArgs& a, int act_dtype, cudaStream_t s) {
+  if (a.batch == 0) return cudaSuccess;
+  dim3 grid(a.batch, a.num_heads);
+  size_t smem = sizeof(float) * a.num_splits;
+  if (act_dtype == MLA_FP32) {
+    combine_kernel<float><<<grid, 128, smem, s>>>(a);
+  } else {
+    combine_kernel<__nv_bfloat16><<<grid, 128, smem, s>>>(a);
+  }
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// output side, dimension-generic: o = W_UV o_lat per head, y = W_O o
+// ---------------------------------------------------------------------------
+
+constexpr int kOpBatch = 32;
+
+// grid (H, ceil(d_v / 8)); warp per output row v; lanes over d_c.
+template <typename T>
+__global__ void __launch_bounds__(256) uv_generic_kernel(OutProjArgs a) {
+  extern __shared__ float ol[];   // [kOpBatch][d_c]
+  const int h = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int v = blockIdx.y * 8 + warp;
+  const T* olat = reinterpret_cast<const T*>(a.o_lat);
+  const T* w = reinterpret_cast<const T*>(a.w_uv) + (static_cast<long>(h) * a.d_v + v) * a.d_c;
+  T* o = reinterpret_cast<T*>(a.o);
+  for (int b0 = 0; b0 < a.batch; b0 += kOpBatch) {
+    const int nb = min(kOpBatch, a.batch - b0);
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < nb * a.d_c; idx += blockDim.x) {
+      const int i = idx / a.d_c, c = idx % a.d_c;
+      ol[idx] = ld_f32(olat, (static_cast<long>(b0 + i) * a.num_heads + h) * a.d_c + c);
+    }
+    __syncthreads();
+    if (v < a.d_v) {
+      float acc[kOpBatch];
+#pragma unroll
+      for (int i = 0; i < kOpBatch; ++i) acc[i] = 0.f;
+      for (int c = lane; c < a.d_c; c += 32) {
+        const float wv = ld_f32(w, c);
+#pragma unroll
+        for (int i = 0; i < kOpBatch; ++i) acc[i] += wv * ol[(i < nb ? i : 0) * a.d_c + c];
+      }
+#pragma unroll
+      for (int i = 0; i < kOpBatch; ++i) {
+        const float r = warp_sum(acc[i]);
+        if (lane == 0 && i < nb)
+          o[(static_cast<long>(b0 + i) * a.num_heads + h) * a.d_v + v] = cvt_out<T>(r);
+      }
+    }
+  }
+}
+
+// grid ceil(d_model / 8); warp per output row m; K = H*d_v streamed in chunks of 256.
+template <typename T>
+__global__ void __launch_bounds__(256) wo_generic_kernel(OutProjArgs a) {
+  __shared__ float os[kOpBatch][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m = blockIdx.x * 8 + warp;
+  const int K = a.num_heads * a.d_v;
+  const T* o = reinterpret_cast<const T*>(a.o);
+  const T* w = reinterpret_cast<const T*>(a.w_o) + static_cast<long>(m) * K;
+  T* y = reinterpret_cast<T*>(a.y);
+  for (int b0 = 0; b0 < a.batch; b0 += kOpBatch) {
+    const int nb = min(kOpBatch, a.batch - b0);
+    float acc[kOpBatch];
+#pragma unroll
+    for (int i = 0; i < kOpBatch; ++i) acc[i] = 0.f;
+    for (int k0 = 0; k0 < K; k0 += 256) {
+      __syncthreads();
+      // os[b][e*32 + l] = o[b][k0 + 8*l + e]
+      for (int idx = threadIdx.x; idx < kOpBatch * 256; idx += blockDim.x) {
+        const int i = idx / 256, r = idx % 256;
+        const int kk = k0 + r;
+        const int l = r / 8, e = r % 8;
+        os[i][e * 32 + l] = (i < nb && kk < K) ? ld_f32(o, static_cast<long>(b0 + i) * K + kk) : 0.f;
+      }
+      __syncthreads();
+      if (m < a.d_model) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int kk = k0 + 8 * lane + e;
+          const float wv = kk < K ? ld_f32(w, kk) : 0.f;
+#pragma unroll
+          for (int i = 0; i < kOpBatch; ++i) acc[i] += wv * os[i][e * 32 + lane];
+        }
+      }
+    }
+    if (m < a.d_model) {
+#pragma unroll
+      for (int i = 0; i < kOpBatch; ++i) {
+        const float r = warp_sum(acc[i]);
+        if (lane == 0 && i < nb) y[static_cast<long>(b0 + i) * a.d_model + m] = cvt_out<T>(r);
+      }
+    }
+  }
+}
+
+cudaError_t launch_out_proj_generic(const OutProjArgs& a, int act_dtype, cudaStream_t s) {
+  if (a.batch == 0) return cudaSuccess;
+  dim3 g1(a.num_heads, (a.d_v + 7) / 8);
+  size_t smem1 = sizeof(float) * kOpBatch * a.d_c;
+  dim3 g2((a.d_model + 7) / 8);
+  if (act_dtype == MLA_FP32) {
+    cudaError_t e = cudaFuncSetAttribute(uv_generic_kernel<float>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+    if (e != cudaSuccess) return e;
+    uv_generic_kernel<float><<<g1, 256, smem1, s>>>(a);
+    wo_generic_kernel<float><<<g2, 256, 0, s>>>(a);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(uv_generic_kernel<__nv_bfloat16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+    if (e != cudaSuccess) return e;
+    uv_generic_kernel<__nv_bfloat16><<<g1, 256, smem1, s>>>(a);
+    wo_generic_kernel<__nv_bfloat16><<<g2, 256, 0, s>>>(a);
+  }
+  note_launches(2);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

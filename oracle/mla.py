@@ -315,8 +315,11 @@ def step_outputs(wl, seqs: Optional[List[int]] = None, fp8_dequant: bool = False
         rows = cache_row(c, k, pos, base)
         if fp8_dequant:
             from .e4m3 import e4m3_decode
-            codes, sc = fp8_quantize_row(rows.astype(np.float32))
-            o, l = decode_absorbed(q_lat[i], e4m3_decode(codes), scale, d["d_c"], row_scale=sc)
+            deq = np.empty_like(rows)
+            for r0 in range(0, rows.shape[0], 8192):     # rows are quantised independently
+                codes, sc = fp8_quantize_row(rows[r0:r0 + 8192].astype(np.float32))
+                deq[r0:r0 + 8192] = e4m3_decode(codes) * sc[:, None].astype(np.float64)
+            o, l = decode_absorbed(q_lat[i], deq, scale, d["d_c"])
         else:
             o, l = decode_absorbed(q_lat[i], rows, scale, d["d_c"])
         o_lat.append(o)

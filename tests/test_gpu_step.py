@@ -1,0 +1,182 @@
+"""GPU parity of a whole decode step (append -> absorb -> split-KV decode ->
+merge -> output projection) through the C ABI, against the fp64 oracle on the
+same seeded inputs.
+
+Small cases span several 64-token pages, several splits and a ragged tail;
+the full-size cases run the workloads at their benchmark sizes in the launch
+configuration the benchmark times and compare sampled sequences (all of them
+where the oracle is cheap)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from helpers import BF16_MAE, BF16_MAX_REL, FP8_MAX_REL, assert_close
+
+pytestmark = pytest.mark.gpu
+
+KEYS = ("q_lat", "o_lat", "lse", "o", "y")
+
+
+def _run(wl, num_splits=0, stage_hook=None):
+    from mla_latent_kv_19_b200.step import DecodeStep
+    st = DecodeStep(wl, num_splits=num_splits)
+    if stage_hook:
+        stage_hook(st)
+    st.run()
+    out = st.outputs()
+    splits = st.num_splits
+    st.close()
+    return out, splits
+
+
+def _compare(wl, g, seqs, tag=""):
+    r = oracle.step_outputs(wl, seqs)
+    fp8 = wl.cache_dtype == "fp8_e4m3"
+    for k in KEYS:
+        lim = FP8_MAX_REL if (fp8 and k != "q_lat") else BF16_MAX_REL
+        assert_close(f"{tag}{k}", g[k][seqs], r[k], max_rel=lim, mae=BF16_MAE)
+    if fp8:
+        # against the oracle run on its own e4m3 rows: the bf16 tolerance
+        rq = oracle.step_outputs(wl, seqs, fp8_dequant=True)
+        for k in ("o_lat", "lse", "o", "y"):
+            assert_close(f"{tag}{k}(dequant)", g[k][seqs], rq[k])
+    return r
+
+
+SMALL = [
+    ("tiny_fp32", {}),
+    ("v2_b32_l2048", dict(batch=3, context=333)),
+    ("v2_b32_l2048_shuf", dict(batch=5, context=1000)),
+    ("v2_ragged64", dict(batch=7, context=900)),
+    ("v2_b4_l32k", dict(batch=2, context=4097)),
+    ("v2_b2_l128k_fp8", dict(batch=2, context=1500)),
+]
+
+
+@pytest.mark.parametrize("name,kw", SMALL, ids=[s[0] + "-small" for s in SMALL])
+def test_step_small(name, kw):
+    wl = workloads.make(name, **kw)
+    g, _ = _run(wl)
+    _compare(wl, g, list(range(wl.batch)))
+
+
+@pytest.mark.parametrize("splits", [1, 2, 5, 16])
+def test_split_count_does_not_change_the_result(splits):
+    wl = workloads.make("v2_b32_l2048", batch=2, context=1100)
+    g, s = _run(wl, num_splits=splits)
+    assert s == splits
+    _compare(wl, g, [0, 1], tag=f"S={splits} ")
+
+
+def test_page_permutation_does_not_change_the_result():
+    a = workloads.make("v2_b32_l2048", batch=4, context=700)
+    b = workloads.make("v2_b32_l2048_shuf", batch=4, context=700)
+    assert not np.array_equal(a.block_table, b.block_table)
+    ga, _ = _run(a, num_splits=3)
+    gb, _ = _run(b, num_splits=3)
+    for k in KEYS:
+        np.testing.assert_array_equal(ga[k], gb[k], err_msg=k)
+
+
+def test_append_then_decode_equals_prefilled_cache():
+    """The decode step's own append (one token per sequence) writes exactly
+    what writing that token together with the history would have written."""
+    from mla_latent_kv_19_b200 import mla_cache_append
+    from mla_latent_kv_19_b200.step import to_device
+    wl = workloads.make("v2_b32_l2048", batch=3, context=200)
+    ga, _ = _run(wl, num_splits=2)
+
+    def prefill_new_tokens(st):
+        seq = to_device(np.arange(wl.batch, dtype=np.int32), "cuda")
+        mla_cache_append(st.h, st.new_c_kv, st.new_k_r, st.new_pos, st.block_table, st.cache,
+                         st.cache_scale, seq_idx=seq, batch=wl.batch)
+        st.append = lambda stream=None: None      # the step itself appends nothing
+    gb, _ = _run(wl, num_splits=2, stage_hook=prefill_new_tokens)
+    for k in KEYS:
+        np.testing.assert_array_equal(ga[k], gb[k], err_msg=k)
+
+
+def test_empty_sequence_gives_zero_and_minus_inf():
+    wl = workloads.make("v2_b32_l2048", batch=3, context=300)
+
+    def empty_middle(st):
+        lens = st.seq_lens.cpu().numpy()
+        lens[1] = 0
+        st.seq_lens.copy_(torch.from_numpy(lens))
+    g, _ = _run(wl, num_splits=2, stage_hook=empty_middle)
+    assert np.all(g["o_lat"][1] == 0)
+    assert np.all(np.isneginf(g["lse"][1]))
+    r = oracle.step_outputs(wl, [0, 2])
+    for k in ("o_lat", "lse"):
+        assert_close(k, g[k][[0, 2]], r[k])
+
+
+def test_combine_against_oracle_merge():
+    from mla_latent_kv_19_b200 import (Handle, mla_decode_combine, mla_decode_workspace_bytes)
+    from mla_latent_kv_19_b200.step import softmax_scale
+    d = workloads.V2_DIMS
+    h = Handle(num_heads=d["num_heads"], d_c=d["d_c"], d_r=d["d_r"], d_nope=d["d_nope"],
+               d_v=d["d_v"], d_model=d["d_model"], softmax_scale=softmax_scale(128, 64),
+               max_position=4096)
+    B, S, H, dc = 3, 6, d["num_heads"], d["d_c"]
+    rng = np.random.default_rng(7)
+    o = rng.standard_normal((B, S, H, dc)).astype(np.float32)
+    lse = (rng.standard_normal((B, S, H)) * 4).astype(np.float32)
+    lse[0, 2] = -np.inf
+    lse[1, :, 5] = -np.inf           # every split of (b=1, h=5) empty
+    o[0, 2] = 0
+    o[1, :, 5] = 0
+    nbytes = mla_decode_workspace_bytes(h, B, S, 64 * S)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    n_o = B * S * H * dc * 4
+    ws[:n_o].view(torch.float32).copy_(torch.from_numpy(o.reshape(-1)))
+    off = (n_o + 255) // 256 * 256
+    ws[off:off + B * S * H * 4].view(torch.float32).copy_(torch.from_numpy(lse.reshape(-1)))
+    o_lat = torch.empty(B, H, dc, dtype=torch.bfloat16, device="cuda")
+    g_lse = torch.empty(B, H, dtype=torch.float32, device="cuda")
+    mla_decode_combine(h, B, 64 * S, S, ws, o_lat, g_lse)
+    ro, rl = oracle.combine(np.moveaxis(o, 1, 0), np.moveaxis(lse, 1, 0))
+    assert_close("o_lat", o_lat.float().cpu().numpy(), ro)
+    gl = g_lse.cpu().numpy()
+    assert np.isneginf(gl[1, 5]) and np.all(o_lat[1, 5].float().cpu().numpy() == 0)
+    assert_close("lse", gl, rl)
+    h.close()
+
+
+# ---------------------------------------------------------------------------
+# full sizes, launch configuration of the benchmark (automatic split count)
+# ---------------------------------------------------------------------------
+
+FULL = ["v2_b32_l2048", "v2_ragged64", "v2_b4_l32k", "v2_b2_l128k_fp8"]
+
+
+def _sample(wl):
+    if wl.name == "v2_ragged64":
+        lens = wl.hist_len
+        return sorted({int(lens.argmax()), int(lens.argmin()), 0, 17, 42, 63})
+    return list(range(wl.batch))
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_step_full_size(name):
+    wl = workloads.make(name)
+    g, _ = _run(wl)
+    seqs = _sample(wl)
+    _compare(wl, g, seqs)
+    # the un-absorbed (primary) form directly, on a few heads of one sequence
+    b = seqs[-1]
+    heads = [0, 77] if wl.seq_lens[b] > 40000 else [0, 31, 77, 127]
+    o_un, lse_un = oracle.mla.step_outputs_unabsorbed(wl, b, heads)
+    lim = FP8_MAX_REL if wl.cache_dtype == "fp8_e4m3" else BF16_MAX_REL
+    assert_close("o(unabsorbed)", g["o"][b, heads], o_un, max_rel=lim)
+    assert_close("lse(unabsorbed)", g["lse"][b, heads], lse_un, max_rel=lim)
+
+
+def test_tiny_fp32_every_output_unabsorbed():
+    wl = workloads.make("tiny_fp32")
+    g, _ = _run(wl)
+    o_un, lse_un = oracle.mla.step_outputs_unabsorbed(wl, 0)
+    assert_close("o", g["o"][0], o_un)
+    assert_close("lse", g["lse"][0], lse_un)
