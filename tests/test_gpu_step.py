@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import workloads
-from helpers import BF16_MAE, BF16_MAX_REL, FP8_MAX_REL, assert_close
+from helpers import BF16_MAE, BF16_MAX_REL, FP8_MAX_REL, assert_close, errors
 
 pytestmark = pytest.mark.gpu
 
@@ -34,12 +34,17 @@ def _run(wl, num_splits=0, stage_hook=None):
 def _compare(wl, g, seqs, tag=""):
     r = oracle.step_outputs(wl, seqs)
     fp8 = wl.cache_dtype == "fp8_e4m3"
+    rq = oracle.step_outputs(wl, seqs, fp8_dequant=True) if fp8 else None
     for k in KEYS:
-        lim = FP8_MAX_REL if (fp8 and k != "q_lat") else BF16_MAX_REL
+        lim = BF16_MAX_REL
+        if fp8 and k != "q_lat":
+            # against exact values the e4m3 rounding of the cache itself counts:
+            # 3e-2, or the oracle's own fp8 error where that is larger (short
+            # contexts average the rounding noise over few tokens)
+            lim = max(FP8_MAX_REL, 1.1 * errors(rq[k], r[k])[0])
         assert_close(f"{tag}{k}", g[k][seqs], r[k], max_rel=lim, mae=BF16_MAE)
     if fp8:
         # against the oracle run on its own e4m3 rows: the bf16 tolerance
-        rq = oracle.step_outputs(wl, seqs, fp8_dequant=True)
         for k in ("o_lat", "lse", "o", "y"):
             assert_close(f"{tag}{k}(dequant)", g[k][seqs], rq[k])
     return r
