@@ -199,6 +199,30 @@ MLA_API int mla_decode_combine(mla_handle_t h, int32_t batch, int32_t max_seq_le
                        const void* workspace, size_t workspace_bytes, void* o_lat, float* lse,
                        cudaStream_t stream);
 
+/* mla_decode_noalloc -- mla_decode for callers that cannot allocate device
+ * memory (for example a plugin inside a framework that owns every device
+ * buffer through its own pool, or a loop that must not risk the implicit
+ * device synchronisation of cudaMalloc).  The pages have no counterpart: this
+ * is a deployment convenience of this library, not a step of the method.
+ *
+ * Same arguments and results as mla_decode minus the workspace: the split
+ * partials go to a 32 MiB array compiled into the library, which stays
+ * allocated on every GPU that loads the library until the process exits.
+ * - A call whose workspace (mla_decode_workspace_bytes for the same batch,
+ *   num_splits and max_seq_len) exceeds 32 MiB returns MLA_ERR_WORKSPACE and
+ *   launches nothing.
+ * - The first call on a device looks up the array's device address (with that
+ *   device current); make that first call before any stream capture.
+ * - Every call on a device shares the one array, which keeps the last call's
+ *   contents; nothing in it needs clearing between calls, but calls that
+ *   overlap on the GPU (other streams, other threads) race on it.
+ * - It calls no cudaMalloc, cudaFree or other allocating routine. */
+MLA_API int mla_decode_noalloc(mla_handle_t h, const void* q_lat, const void* cache,
+                               const float* cache_scale, int32_t num_blocks,
+                               const int32_t* block_table, int32_t max_blocks_per_seq,
+                               const int32_t* seq_lens, int32_t batch, int32_t max_seq_len,
+                               int32_t num_splits, void* o_lat, float* lse, cudaStream_t stream);
+
 /* Workspace bytes mla_out_proj needs for this batch. */
 MLA_API size_t mla_out_proj_workspace_bytes(mla_handle_t h, int32_t batch);
 

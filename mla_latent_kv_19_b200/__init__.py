@@ -19,6 +19,7 @@ __all__ = [
     "MLAError", "Handle", "lib", "LIB_PATH",
     "mla_create", "mla_destroy", "mla_cache_append", "mla_kv_project_append", "mla_absorb_q",
     "mla_decode", "mla_decode_partial", "mla_decode_combine", "mla_decode_auto_splits",
+    "mla_decode_noalloc",
     "mla_decode_workspace_bytes", "mla_out_proj", "mla_out_proj_workspace_bytes",
     "mla_last_device_error", "mla_set_wait_limit", "mla_status_string", "mla_launch_count",
     "MLA_BF16", "MLA_FP8_E4M3", "MLA_FP32", "EXPORTED_SYMBOLS",
@@ -63,6 +64,7 @@ _SIGS = {
     "mla_decode": (ctypes.c_int, [_P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _P, _SZ, _P, _P, _P]),
     "mla_decode_partial": (ctypes.c_int, [_P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _P, _SZ, _P]),
     "mla_decode_combine": (ctypes.c_int, [_P, _I, _I, _I, _P, _SZ, _P, _P, _P]),
+    "mla_decode_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _P, _P, _P]),
     "mla_out_proj_workspace_bytes": (_SZ, [_P, _I]),
     "mla_out_proj": (ctypes.c_int, [_P, _P, _P, _P, _I, _P, _SZ, _P, _P, _P]),
     "mla_last_device_error": (ctypes.c_int, [_P, _P]),
@@ -200,6 +202,17 @@ def mla_decode_combine(h: Handle, batch: int, max_seq_len: int, num_splits: int,
     _check("mla_decode_combine", lib.mla_decode_combine(
         h.ptr, batch, max_seq_len, num_splits, _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(o_lat), _ptr(lse), _stream(stream)))
+
+
+def mla_decode_noalloc(h: Handle, q_lat, cache, cache_scale, block_table, seq_lens,
+                       max_seq_len: int, num_splits: int, o_lat, lse=None, stream=None) -> None:
+    """mla_decode without a caller workspace: the split partials live in a
+    fixed 32 MiB device array inside the library (for callers that cannot
+    allocate device memory).  Overlapping calls on one device race on it."""
+    _check("mla_decode_noalloc", lib.mla_decode_noalloc(
+        h.ptr, _ptr(q_lat), _ptr(cache), _ptr(cache_scale), cache.shape[0], _ptr(block_table),
+        block_table.shape[1], _ptr(seq_lens), seq_lens.shape[0], max_seq_len, num_splits,
+        _ptr(o_lat), _ptr(lse), _stream(stream)))
 
 
 def mla_out_proj_workspace_bytes(h: Handle, batch: int) -> int:
