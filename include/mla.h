@@ -188,8 +188,9 @@ MLA_API int mla_decode(mla_handle_t h, const void* q_lat, const void* cache, con
 /* The two halves of mla_decode, for callers that time or schedule them
  * separately.  mla_decode_partial writes the workspace; mla_decode_combine
  * reads it (same batch / num_splits / max_seq_len) and writes o_lat and lse.
- * Workspace layout (fp32): o_part [batch][S][H][d_c] followed by
- * lse_part [batch][S][H]; an empty range stores lse_part = -inf, o_part = 0. */
+ * Workspace layout (fp32): o_part [batch][S][d_c][H] (heads innermost) followed,
+ * at the next 256-byte boundary, by lse_part [batch][S][H]; an empty range
+ * stores lse_part = -inf, o_part = 0. */
 MLA_API int mla_decode_partial(mla_handle_t h, const void* q_lat, const void* cache,
                        const float* cache_scale, int32_t num_blocks, const int32_t* block_table,
                        int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t batch,

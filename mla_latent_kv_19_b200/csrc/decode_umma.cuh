@@ -14,16 +14,27 @@
 // page does not leave room for a pipeline in one SM's shared memory.  A
 // cluster of two CTAs splits the roles:
 //
-//   CTA 0 ("score"):  Q lives in TMEM (columns 0..287, two bf16 per column)
-//     and is the A operand of TS-form UMMAs; pages stream through a 3-stage
-//     TMA ring; S = Q K^T goes to one of two TMEM buffers (columns 384/448);
-//     four softmax warps (one TMEM lane quadrant each, one head per thread)
-//     run the online softmax and store P (bf16, UMMA K-major 128B-swizzled
-//     layout) straight into CTA 1's shared memory.
+//   CTA 0 ("score"):  a ring of 3 shared-memory slots of 72 KB, each filled
+//     by ONE 3-D TMA request that lands a whole page (64 rows x 576 columns)
+//     as 9 column chunks of [64 rows x 128 bytes] with the 128-byte swizzle
+//     (the UMMA K-major layout); the first two slots carry Q (two halves of
+//     64 heads) into TMEM (columns 0..287, two bf16 per column; Q is then the
+//     A operand of TS-form UMMAs); S = Q K^T (N = 64, one page per MMA) goes
+//     to one of two TMEM buffers (columns 384/448); four softmax warps (one
+//     TMEM lane quadrant each, one head per thread) run the online softmax and
+//     write P (bf16, UMMA K-major swizzled layout) plus the rescale factors
+//     into the page's own slot -- its K data is no longer needed -- and one
+//     thread ships that message to CTA 1 with a single bulk copy; CTA 1 frees
+//     the slot once its P V has consumed the message.
 //   CTA 1 ("value"):  O accumulates in TMEM columns 0..511; the same pages'
-//     first 512 columns stream through a 2-stage TMA ring (an L2 hit after
-//     CTA 0's read); P V is issued as two N = 256 SS-form UMMAs per 16-token
-//     K step, V being the MN-major B operand.
+//     first 512 columns stream through a 2-stage ring, one 64 KB TMA request
+//     per page (an L2 hit after CTA 0's read); P V is issued as two N = 256
+//     SS-form UMMAs per 16-token K step, V being the MN-major B operand.
+//
+// Measured on B200: issuing a TMA request costs the producer a few hundred
+// cycles (so requests are whole pages), and a tcgen05.mma with M = 128 costs
+// at least ~60 cycles whatever its N up to 128 (so S takes a full page, N = 64,
+// per instruction rather than half pages).
 //
 // The running maximum is only moved when a tile's maximum exceeds it by more
 // than 8 (log2 units), so P stays <= 256 and O needs rescaling (a TMEM read-
@@ -42,32 +53,44 @@ namespace mla {
 namespace dec {
 
 constexpr int kH = 128, kDc = 512, kD = 576, kTok = 64;
-constexpr int kBoxBytes = 64 * 128;                    // 64 rows x 64 bf16
-constexpr int kKBoxes = 9, kVBoxes = 8;
-constexpr int kKStageBytes = kKBoxes * kBoxBytes;      // 73728
+constexpr int kBoxBytes = 64 * 128;                    // 64 rows x 64 bf16 (one column chunk)
+constexpr int kKBoxes = 9, kVBoxes = 8;                // column chunks of a row / of V
+constexpr int kSlotBytes = kKBoxes * kBoxBytes;        // 73728: 9 chunks x 64 rows x 128 B
+constexpr int kChunkInSlot = kBoxBytes;                // 8192
+constexpr int kQLoads = 2;                             // two halves of 64 heads
+constexpr int kSlots = 3;                              // CTA 0 ring
 constexpr int kVStageBytes = kVBoxes * kBoxBytes;      // 65536
-constexpr int kKStages = 3, kVStages = 2;
+constexpr int kVStages = 2;
 constexpr int kPBytes = kH * kTok * 2;                 // 16384
+constexpr int kPMsgBytes = kPBytes + kH * 4 + 16;      // P + alpha[128] + flag[4] = 16912
+constexpr int kPBufStride = 17 * 1024;                 // keeps every P tile 1024-byte aligned
+constexpr int kMaxTablePages = 512;                    // pages of a split kept in shared memory
 
-// shared-memory map, offsets from a 1024-byte aligned base
-constexpr int kOffK = 0;                               // CTA 0: K ring
-constexpr int kOffV = 0;                               // CTA 1: V ring
-constexpr int kOffP = kVStages * kVStageBytes;         // CTA 1: P[2]
-constexpr int kOffAlpha = kOffP + 2 * kPBytes;         // CTA 1: alpha[2][128]
-constexpr int kOffFlag = kOffAlpha + 2 * kH * 4;       // CTA 1: flag[2][4]
-constexpr int kOffLfin = kOffFlag + 2 * 4 * 4;         // CTA 1: l[128]
-constexpr int kRegionEnd = kKStages * kKStageBytes;    // 221184
-static_assert(kOffLfin + kH * 4 <= kRegionEnd, "CTA 1 buffers overlap the barriers");
+// CTA 0 map
+constexpr int kOffRing = 0;
+constexpr int kOffTable0 = kSlots * kSlotBytes;        // 221184
+// CTA 1 map
+constexpr int kOffV = 0;
+constexpr int kPBufs = kSlots;                         // message t lives in buffer t % 3
+constexpr int kOffP = kVStages * kVStageBytes;         // 131072: P messages [3]
+constexpr int kOffLfin = kOffP + kPBufs * kPBufStride; // l[128]
+constexpr int kOffTable1 = kOffLfin + kH * 4;
+constexpr int kRegionEnd = kOffTable0 + kMaxTablePages * 4;
+static_assert(kOffTable1 + kMaxTablePages * 4 <= kRegionEnd, "CTA 1 map overlaps the barriers");
 
 enum Bar {
-  kKFull = 0, kKEmpty = 3, kSFull = 6, kSEmpty = 8, kPEmpty = 10, kQReady = 12,  // CTA 0
-  kVFull = 13, kVEmpty = 15, kPFull = 17, kPVDone = 19, kCorrReq = 21,           // CTA 1
-  kCorrDone = 22, kOFull = 23, kFin = 24,
-  kDrain = 25, kNumBars = 26
+  kFull = 0, kEmpty = kFull + kSlots,                                     // CTA 0 ring
+  kSFull = kEmpty + kSlots, kSEmpty = kSFull + 2,                        // CTA 0
+  kQReady = kSEmpty + 2, kStg = kQReady + 1,
+  kVFull = kStg + 2, kVEmpty = kVFull + kVStages,                       // CTA 1
+  kPFull = kVEmpty + kVStages, kPVDone = kPFull + kPBufs,
+  kCorrReq = kPVDone + 2, kCorrDone = kCorrReq + 1, kOFull = kCorrDone + 1, kFin = kOFull + 1,
+  kDrain = kFin + 1, kNumBars = kDrain + 1
 };
 constexpr int kOffBar = kRegionEnd;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;       // [0] tmem base, [1] abort, [2] corr tile
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;       // + slack for the 1024-byte alignment
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
@@ -104,21 +127,23 @@ __device__ __forceinline__ Split split_of(const DecodeArgs& a, int pair, int* er
   return s;
 }
 
-// Physical page of tile t and its number of valid tokens (0 for an invalid page,
-// which is then read from page 0 and masked entirely).
-__device__ __forceinline__ int tile_page(const DecodeArgs& a, const Split& s, int t, int* valid) {
-  const int idx = s.p0 + t;
-  const int pg = a.block_table[static_cast<long>(s.b) * a.max_blocks + idx];
-  if (pg < 0 || pg >= a.num_blocks) {
-    *valid = 0;
-    return -1;
-  }
-  *valid = min(kTok, s.len - idx * kTok);
-  return pg;
+// Physical page of tile t (-1 if the table entry is outside the pool).
+__device__ __forceinline__ int load_page(const DecodeArgs& a, const Split& s, int t) {
+  const int pg = a.block_table[static_cast<long>(s.b) * a.max_blocks + s.p0 + t];
+  return (pg < 0 || pg >= a.num_blocks) ? -1 : pg;
+}
+
+__device__ __forceinline__ int page_at(const DecodeArgs& a, const Split& s, const int* table, int t) {
+  return t < kMaxTablePages ? table[t] : load_page(a, s, t);
+}
+
+__device__ __forceinline__ int valid_tokens(const Split& s, int page, int t) {
+  return page < 0 ? 0 : min(kTok, s.len - (s.p0 + t) * kTok);
 }
 
 __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
-    decode_umma_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
+    decode_umma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                       const __grid_constant__ CUtensorMap qmap, const DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -133,7 +158,6 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
   const Split sp = split_of(a, static_cast<int>(blockIdx.x >> 1), &bad_len);
   if (bad_len && threadIdx.x == 0 && rank == 0) report_error(a.err, MLA_ERR_BAD_INDEX);
 
-  // bounded waits; a warp-uniform verdict, and the abort flag on failure
   auto fail = [&]() {
     misc[1] = 1u;
     report_error(a.err, MLA_ERR_TIMEOUT);
@@ -152,26 +176,29 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
   };
   auto drain = [&](uint32_t b_, uint32_t par) { ptx::mbar_wait<false>(b_, par, kDrainIters, kWaitNs); };
 
+  // this split's page table, kept in shared memory
+  int* table = reinterpret_cast<int*>(smem + (rank == 0 ? kOffTable0 : kOffTable1));
+  for (int t = threadIdx.x; t < min(sp.ntiles, kMaxTablePages); t += blockDim.x) {
+    const int pg = load_page(a, sp, t);
+    table[t] = pg;
+    if (pg < 0 && rank == 0) report_error(a.err, MLA_ERR_BAD_INDEX);
+  }
   if (threadIdx.x == 0) {
-    // CTA 0
-    for (int i = 0; i < kKStages; ++i) {
-      ptx::mbar_init(bar(kKFull + i), 1);
-      ptx::mbar_init(bar(kKEmpty + i), 1);
+    for (int i = 0; i < kSlots; ++i) {
+      ptx::mbar_init(bar(kFull + i), 1);
+      ptx::mbar_init(bar(kEmpty + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(bar(kSFull + i), 1);
       ptx::mbar_init(bar(kSEmpty + i), 128);
-      ptx::mbar_init(bar(kPEmpty + i), 1);
+      ptx::mbar_init(bar(kPVDone + i), 1);
+      ptx::mbar_init(bar(kStg + i), 128);
     }
+    for (int i = 0; i < kPBufs; ++i) ptx::mbar_init(bar(kPFull + i), 1);
     ptx::mbar_init(bar(kQReady), 128);
-    // CTA 1
     for (int i = 0; i < kVStages; ++i) {
       ptx::mbar_init(bar(kVFull + i), 1);
       ptx::mbar_init(bar(kVEmpty + i), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(bar(kPFull + i), 128);
-      ptx::mbar_init(bar(kPVDone + i), 1);
     }
     ptx::mbar_init(bar(kCorrReq), 1);
     ptx::mbar_init(bar(kCorrDone), 128);
@@ -182,6 +209,7 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
     misc[2] = 0u;
     ptx::fence_mbar_init_cluster();
   }
+  __syncwarp();
   if (warp == 1) {
     ptx::tmem_alloc(sb + kOffMisc, kTmemCols);
     ptx::tmem_relinquish();
@@ -194,46 +222,57 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
 
   if (rank == 0) {
     // =========================== CTA 0: scores and softmax ===========================
-    if (warp == 0 && lane == 0) {
-      // TMA producer: full 576-column pages
-      ptx::prefetch_tmap(&tmap);
-      int issued = 0;
-      for (int t = 0; t < sp.ntiles; ++t) {
-        const int st = t % kKStages;
-        if (!wait_local(bar(kKEmpty + st), ((t / kKStages) & 1) ^ 1)) break;
-        int valid;
-        int pg = tile_page(a, sp, t, &valid);
-        if (pg < 0) {
-          report_error(a.err, MLA_ERR_BAD_INDEX);
-          pg = 0;
-        }
-        ptx::mbar_arrive_expect_tx(bar(kKFull + st), kKStageBytes);
-        const uint32_t dst = sb + kOffK + st * kKStageBytes;
-        for (int i = 0; i < kKBoxes; ++i)
-          ptx::tma_load_2d(dst + i * kBoxBytes, &tmap, bar(kKFull + st), i * 64, pg * kTok);
-        issued = t + 1;
-      }
-      for (int t = max(0, issued - kKStages); t < issued; ++t)
-        drain(bar(kKFull + t % kKStages), (t / kKStages) & 1);
-    } else if (warp == 1) {
-      // MMA issuer: S[i] = Q K^T, A = Q from TMEM, B = page from shared memory
+    if (warp == 0) {
       if (lane == 0) {
-        constexpr uint32_t idS = ptx::idesc_bf16_f32(128, 64, false, false);
+        // TMA producer over the ring: 2 halves of Q, then one request per page.  A
+        // page's slot comes back when CTA 1 has consumed the P message in it.
+        ptx::prefetch_tmap(&kmap);
+        ptx::prefetch_tmap(&qmap);
+        const int total = kQLoads + sp.ntiles;
+        int issued = 0;
+        for (int n = 0; n < total; ++n) {
+          const int slot = n % kSlots;
+          if (!wait_remote(bar(kEmpty + slot), ((n / kSlots) & 1) ^ 1)) break;
+          ptx::mbar_arrive_expect_tx(bar(kFull + slot), kSlotBytes);
+          const uint32_t dst = sb + kOffRing + slot * kSlotBytes;
+          if (n < kQLoads) {
+            ptx::tma_load_3d(dst, &qmap, bar(kFull + slot), 0, sp.b * kH + 64 * n, 0);
+          } else {
+            const int pg = page_at(a, sp, table, n - kQLoads);
+            ptx::tma_load_3d(dst, &kmap, bar(kFull + slot), 0, (pg < 0 ? 0 : pg) * kTok, 0);
+          }
+          issued = n + 1;
+        }
+        for (int n = max(0, issued - kSlots); n < issued; ++n)
+          drain(bar(kFull + n % kSlots), (n / kSlots) & 1);
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      // MMA issuer: S[i] = Q K^T, A = Q from TMEM, B = page boxes from the ring
+      if (lane == 0) {
+        constexpr uint32_t idS = ptx::idesc_bf16_f32(128, kTok, false, false);
         if (wait_local(bar(kQReady), 0)) {
+          for (int n = 0; n < kQLoads; ++n) ptx::mbar_arrive(bar(kEmpty + n));   // Q is in TMEM
+#pragma unroll 1
           for (int t = 0; t < sp.ntiles; ++t) {
-            const int st = t % kKStages, i = t & 1;
-            if (!wait_local(bar(kKFull + st), (t / kKStages) & 1)) break;
+            const int i = t & 1;
+            const int n = kQLoads + t;
+            const int slot = n % kSlots;
             if (!wait_local(bar(kSEmpty + i), ((t >> 1) & 1) ^ 1)) break;
+            if (!wait_local(bar(kFull + slot), (n / kSlots) & 1)) break;
             ptx::tc_fence_after();
+            // S[i] = Q K^T over the 9 chunks of K = 576, one page (N = 64) per MMA
             const uint32_t d = tmem + kColS + 64u * i;
-            const uint32_t kb = sb + kOffK + st * kKStageBytes;
-#pragma unroll 4
-            for (int j = 0; j < kD / 16; ++j) {
-              const uint64_t bd = ptx::sdesc_sw128(kb + (j >> 2) * kBoxBytes + (j & 3) * 32, 16, 1024);
-              ptx::umma_ts(d, tmem + kColQ + 8u * j, bd, idS, j > 0 ? 1u : 0u);
+            const uint32_t kb = sb + kOffRing + slot * kSlotBytes;
+#pragma unroll 3
+            for (int c = 0; c < kKBoxes; ++c) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint64_t bd = ptx::sdesc_sw128(kb + c * kChunkInSlot + j * 32, 16, 1024);
+                ptx::umma_ts(d, tmem + kColQ + 32u * c + 8u * j, bd, idS, (c | j) ? 1u : 0u);
+              }
             }
             ptx::umma_commit(bar(kSFull + i));
-            ptx::umma_commit(bar(kKEmpty + st));
           }
         }
         ptx::umma_commit(bar(kDrain));
@@ -245,40 +284,43 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
       const int q = warp & 3;
       const int r = q * 32 + lane;
       const uint32_t lb = static_cast<uint32_t>(q * 32) << 16;
-      // Q (this sequence's 128 x 576 absorbed queries) -> TMEM, two bf16 per column
-      {
-        const uint4* qrow = reinterpret_cast<const uint4*>(
-            reinterpret_cast<const __nv_bfloat16*>(a.q_lat) + (static_cast<long>(sp.b) * kH + r) * kD);
+      // Q half q/2 (ring slot q/2) holds this warp's 32 heads as 9 column chunks
+      // of 64 rows; the MMA warp frees the slots once every thread has arrived
+      // on q_ready
+      bool ok = wait_local(bar(kFull + (q >> 1)), 0);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        const int row = r & 63;
+        const uint8_t* base = smem + kOffRing + (q >> 1) * kSlotBytes + row * 128;
 #pragma unroll 1
-        for (int c = 0; c < kD / 64; ++c) {
+        for (int c = 0; c < kKBoxes; ++c) {
           uint32_t v[32];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint4 u = __ldg(qrow + c * 8 + k);
-            v[4 * k] = u.x;
-            v[4 * k + 1] = u.y;
-            v[4 * k + 2] = u.z;
-            v[4 * k + 3] = u.w;
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint4 u = *reinterpret_cast<const uint4*>(base + c * kChunkInSlot + ((ch ^ (row & 7)) << 4));
+            v[4 * ch] = u.x;
+            v[4 * ch + 1] = u.y;
+            v[4 * ch + 2] = u.z;
+            v[4 * ch + 3] = u.w;
           }
           ptx::tmem_st32(tmem + lb + kColQ + 32u * c, v);
         }
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(bar(kQReady));
       }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar(kQReady));
+
       const uint32_t rP = ptx::mapa(sb + kOffP, 1);
-      const uint32_t rAlpha = ptx::mapa(sb + kOffAlpha, 1);
-      const uint32_t rFlag = ptx::mapa(sb + kOffFlag, 1);
       const uint32_t rL = ptx::mapa(sb + kOffLfin, 1);
       const uint32_t rPFull = ptx::mapa(bar(kPFull), 1);
       const uint32_t rFin = ptx::mapa(bar(kFin), 1);
       const float sl2 = a.scale * kLog2e;
       float m_used = -INFINITY, l = 0.f;
 #pragma unroll 1
-      for (int t = 0; t < sp.ntiles; ++t) {
+      for (int t = 0; t < sp.ntiles && ok; ++t) {
         const int i = t & 1;
-        bool ok = wait_local(bar(kSFull + i), (t >> 1) & 1);
-        if (!__all_sync(0xffffffffu, ok)) break;
+        bool w = wait_local(bar(kSFull + i), (t >> 1) & 1);
+        if (!__all_sync(0xffffffffu, w)) break;
         ptx::tc_fence_after();
         uint32_t s0[32], s1[32];
         ptx::tmem_ld32(tmem + lb + kColS + 64u * i, s0);
@@ -286,8 +328,7 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
         ptx::tmem_wait_ld();
         ptx::tc_fence_before();
         ptx::mbar_arrive(bar(kSEmpty + i));
-        int valid;
-        tile_page(a, sp, t, &valid);
+        const int valid = valid_tokens(sp, page_at(a, sp, table, t), t);
         float x[64];
         float m_tile = -INFINITY;
 #pragma unroll
@@ -299,7 +340,7 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
         const bool resc = m_tile > m_used + kRescaleThreshold;
         float alpha = 1.f;
         if (resc) {
-          alpha = (m_used == -INFINITY) ? 0.f : exp2f(m_used - m_tile);
+          alpha = (m_used == -INFINITY) ? 0.f : ptx::ex2(m_used - m_tile);
           m_used = m_tile;
         }
         uint32_t pk[32];
@@ -307,26 +348,32 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
         const bool live = m_used != -INFINITY;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float p0 = live ? exp2f(x[2 * j] - m_used) : 0.f;
-          const float p1 = live ? exp2f(x[2 * j + 1] - m_used) : 0.f;
+          const float p0 = live ? ptx::ex2(x[2 * j] - m_used) : 0.f;
+          const float p1 = live ? ptx::ex2(x[2 * j + 1] - m_used) : 0.f;
           const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
           psum += __low2float(pb) + __high2float(pb);
           pk[j] = *reinterpret_cast<const uint32_t*>(&pb);
         }
         l = l * alpha + psum;
-        ok = wait_remote(bar(kPEmpty + i), ((t >> 1) & 1) ^ 1);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        // P row r into CTA 1: 8 chunks of 16 bytes, chunk index xor (row mod 8)
-        const uint32_t prow = rP + i * kPBytes + r * 128;
+        // the message goes into this page's ring slot: S(t) has consumed its K data
+        const int slot = (kQLoads + t) % kSlots;
+        uint8_t* msg = smem + kOffRing + slot * kSlotBytes;
+        uint8_t* prow = msg + r * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-          ptx::st_cluster_v4(prow + ((c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
-                             pk[4 * c + 3]);
-        ptx::st_cluster_u32(rAlpha + (i * kH + r) * 4, __float_as_uint(alpha));
+          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        reinterpret_cast<float*>(msg + kPBytes)[r] = alpha;
         const unsigned any = __any_sync(0xffffffffu, resc && t > 0);
-        if (lane == 0) ptx::st_cluster_u32(rFlag + (i * 4 + q) * 4, any);
-        ptx::fence_proxy_async_cluster();
-        ptx::mbar_arrive_remote(rPFull + 8u * i);
+        if (lane == 0) reinterpret_cast<uint32_t*>(msg + kPBytes + kH * 4)[q] = any;
+        ptx::fence_proxy_async_cta();              // generic writes -> bulk-copy reads
+        ptx::mbar_arrive(bar(kStg + i));
+        if (r == 0) {
+          // every row of the message is written: ship it to CTA 1 in one bulk copy
+          if (wait_local(bar(kStg + i), (t >> 1) & 1))
+            ptx::bulk_copy_to_peer(rP + (t % kPBufs) * kPBufStride, sb + kOffRing + slot * kSlotBytes,
+                                   kPMsgBytes, rPFull + 8u * (t % kPBufs));
+        }
       }
       // this split's log-sum-exp (natural log) and the normaliser for CTA 1
       const long row = (static_cast<long>(sp.b) * a.num_splits + sp.split) * kH + r;
@@ -336,36 +383,36 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
     }
   } else {
     // =========================== CTA 1: values ===========================
-    if (warp == 0 && lane == 0) {
-      // TMA producer: first 512 columns of the same pages
-      ptx::prefetch_tmap(&tmap);
-      int issued = 0;
-      for (int t = 0; t < sp.ntiles; ++t) {
-        const int st = t % kVStages;
-        if (!wait_local(bar(kVEmpty + st), ((t / kVStages) & 1) ^ 1)) break;
-        int valid;
-        int pg = tile_page(a, sp, t, &valid);
-        if (pg < 0) pg = 0;
-        ptx::mbar_arrive_expect_tx(bar(kVFull + st), kVStageBytes);
-        const uint32_t dst = sb + kOffV + st * kVStageBytes;
-        for (int i = 0; i < kVBoxes; ++i)
-          ptx::tma_load_2d(dst + i * kBoxBytes, &tmap, bar(kVFull + st), i * 64, pg * kTok);
-        issued = t + 1;
+    if (warp == 0) {
+      if (lane == 0) {
+        // TMA producer: first 512 columns of the same pages
+        ptx::prefetch_tmap(&vmap);
+        int issued = 0;
+        for (int t = 0; t < sp.ntiles; ++t) {
+          const int st = t % kVStages;
+          if (!wait_local(bar(kVEmpty + st), ((t / kVStages) & 1) ^ 1)) break;
+          const int pg = page_at(a, sp, table, t);
+          ptx::mbar_arrive_expect_tx(bar(kVFull + st), kVStageBytes);
+          ptx::tma_load_3d(sb + kOffV + st * kVStageBytes, &vmap, bar(kVFull + st), 0,
+                           (pg < 0 ? 0 : pg) * kTok, 0);
+          issued = t + 1;
+        }
+        for (int t = max(0, issued - kVStages); t < issued; ++t)
+          drain(bar(kVFull + t % kVStages), (t / kVStages) & 1);
       }
-      for (int t = max(0, issued - kVStages); t < issued; ++t)
-        drain(bar(kVFull + t % kVStages), (t / kVStages) & 1);
+      __syncwarp();
     } else if (warp == 1) {
       // MMA issuer: O += P V  (A = P, K-major; B = V, MN-major; two N = 256 halves)
       constexpr uint32_t idPV = ptx::idesc_bf16_f32(128, 256, false, true);
       int ncorr = 0;
 #pragma unroll 1
       for (int t = 0; t < sp.ntiles; ++t) {
-        const int st = t & 1;
+        const int st = t & 1, pbi = t % kPBufs;
+        if (lane == 0) ptx::mbar_arrive_expect_tx(bar(kPFull + pbi), kPMsgBytes);
         bool ok = wait_local(bar(kVFull + st), (t >> 1) & 1);
-        ok = ok && wait_remote(bar(kPFull + st), (t >> 1) & 1);
+        ok = ok && wait_remote(bar(kPFull + pbi), (t / kPBufs) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
-        int valid;
-        tile_page(a, sp, t, &valid);
+        const int valid = valid_tokens(sp, page_at(a, sp, table, t), t);
         if (valid < kTok) {
           // rows past the sequence end: zero them so that P = 0 meets finite V
           uint8_t* vs = smem + kOffV + st * kVStageBytes;
@@ -378,7 +425,8 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
           ptx::fence_proxy_async_cta();
           __syncwarp();
         }
-        const volatile uint32_t* fl = reinterpret_cast<const volatile uint32_t*>(smem + kOffFlag) + st * 4;
+        const uint8_t* msg = smem + kOffP + pbi * kPBufStride;
+        const uint32_t* fl = reinterpret_cast<const uint32_t*>(msg + kPBytes + kH * 4);
         const uint32_t flag = fl[0] | fl[1] | fl[2] | fl[3];
         if (flag) {
           if (lane == 0) {
@@ -391,8 +439,7 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
         }
         ptx::tc_fence_after();
         if (lane == 0) {
-          ptx::fence_proxy_async_cta();
-          const uint32_t pb = sb + kOffP + st * kPBytes;
+          const uint32_t pb = sb + kOffP + pbi * kPBufStride;
           const uint32_t vb = sb + kOffV + st * kVStageBytes;
 #pragma unroll
           for (int j = 0; j < kTok / 16; ++j) {
@@ -415,21 +462,24 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
         drain(bar(kDrain), 0);
       }
       __syncwarp();
-    } else if (warp == 2 && lane == 0) {
-      // release: a finished P V frees its V stage here and its P buffer's producer in CTA 0
-      const uint32_t rPEmpty = ptx::mapa(bar(kPEmpty), 0);
-      for (int t = 0; t < sp.ntiles; ++t) {
-        const int i = t & 1;
-        if (!wait_local(bar(kPVDone + i), (t >> 1) & 1)) break;
-        ptx::mbar_arrive(bar(kVEmpty + i));
-        ptx::mbar_arrive_remote(rPEmpty + 8u * i);
+    } else if (warp == 2) {
+      // release: a finished P V frees its V stage here and, in CTA 0, the ring
+      // slot that carried its P message
+      if (lane == 0) {
+        const uint32_t rEmpty = ptx::mapa(bar(kEmpty), 0);
+        for (int t = 0; t < sp.ntiles; ++t) {
+          const int i = t & 1;
+          if (!wait_local(bar(kPVDone + i), (t >> 1) & 1)) break;
+          ptx::mbar_arrive(bar(kVEmpty + i));
+          ptx::mbar_arrive_remote(rEmpty + 8u * ((kQLoads + t) % kSlots));
+        }
       }
+      __syncwarp();
     } else if (warp >= 4) {
       // correction (rescale O rows on request) and epilogue
       const int q = warp & 3;
       const int r = q * 32 + lane;
       const uint32_t lb = static_cast<uint32_t>(q * 32) << 16;
-      const float* alphas = reinterpret_cast<const float*>(smem + kOffAlpha);
       int k = 0;
 #pragma unroll 1
       while (true) {
@@ -443,7 +493,8 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
           if (!__all_sync(0xffffffffu, ok)) break;
         }
         ptx::tc_fence_after();
-        const float al = alphas[(t & 1) * kH + r];
+        const float al =
+            reinterpret_cast<const float*>(smem + kOffP + (t % kPBufs) * kPBufStride + kPBytes)[r];
 #pragma unroll 1
         for (int c = 0; c < 16; ++c) {
           uint32_t v[32];
@@ -460,14 +511,14 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
       bool ok = wait_local(bar(kOFull), 0);
       ok = ok && wait_remote(bar(kFin), 0);
       ok = __all_sync(0xffffffffu, ok);
-      float* orow = a.o_part + ((static_cast<long>(sp.b) * a.num_splits + sp.split) * kH + r) * kDc;
+      // o_part[b][split][c][h]: for each column c the 32 lanes store 32 consecutive heads
+      float* obase = a.o_part + (static_cast<long>(sp.b) * a.num_splits + sp.split) * kDc * kH + r;
       if (ok) {
         ptx::tc_fence_after();
         const float lsum = reinterpret_cast<const volatile float*>(smem + kOffLfin)[r];
         const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
         if (sp.ntiles == 0) {
-          for (int c = 0; c < kDc; c += 4)
-            *reinterpret_cast<float4*>(orow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int c = 0; c < kDc; ++c) obase[c * kH] = 0.f;
         } else {
 #pragma unroll 1
           for (int c = 0; c < 16; ++c) {
@@ -475,10 +526,7 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
             ptx::tmem_ld32(tmem + lb + kColO + 32u * c, v);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4*>(orow + 32 * c + e) =
-                  make_float4(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv,
-                              __uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv);
+            for (int e = 0; e < 32; ++e) obase[(32 * c + e) * kH] = __uint_as_float(v[e]) * inv;
           }
         }
         ptx::tc_fence_before();
@@ -486,6 +534,7 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
     }
   }
 
+  __syncwarp();
   __syncthreads();
   ptx::cluster_sync();       // no remote access to this CTA's shared memory after this point
   if (warp == 1) {

@@ -1,0 +1,229 @@
+// Weight-streaming GEMM on tcgen05 tensor cores for the projections around
+// the decode (batch of B <= 256 decode tokens against large bf16 weights):
+//
+//   D[m][b] = sum_k A[m][k] * X[b][k]
+//
+// with the weight as the M operand (128 rows per CTA, "swap-AB": the batch is
+// the N dimension, 16 <= N <= 256) and fp32 accumulation in TMEM.  Uses:
+//   * W_O   (V2 page section 2.3, W_UV absorbed into W_O; applied as W_O after
+//            W_UV):  A = W_O [5120][16384] K-major, X = o [B][16384];
+//            K split over CTAs, fp32 partials reduced by a second kernel.
+//   * W_UV  per head:  A = W_UV[h] [128][512] K-major, X = o_lat[:, h, :].
+//   * W_UK  per head (absorbed query, V2 page section 2.3):  A = W_UK[h]^T,
+//            i.e. W_UK[h] [128][512] read MN-major, X = q_nope[:, h, :];
+//            the epilogue also applies RoPE to q_pe (section 2.2).
+//
+// The kernel is HBM-bound on the weight stream (2 flops per weight byte per
+// token of the batch); a TMA ring of (A, X) chunks of 64 along K keeps enough
+// bytes in flight per SM, one thread issues the UMMAs, four warps drain TMEM.
+#pragma once
+
+#include "device_common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace mla {
+namespace gemm {
+
+constexpr int kM = 128;          // weight rows per CTA
+constexpr int kKc = 64;          // K per pipeline stage (one 128-byte swizzle row of bf16)
+constexpr uint64_t kWaitNs = 1000000000ull;
+
+enum class Epi : int { kStoreBf16T = 0, kPartialF32 = 1, kAbsorb = 2 };
+
+struct Params {
+  int n;                 // padded batch (multiple of 16), the UMMA N
+  int batch;             // real batch
+  int k_chunks;          // K / 64 per group
+  int k_split;           // CTAs along K (gridDim.y)
+  int m_per_group;       // weight rows of one group (head), multiple of 128
+  // A coordinates: K-major: row = group*a_row_group + m, col = k
+  //                MN-major: row = group*a_row_group + k, col = m
+  int a_row_group;
+  // X coordinates: row = b, col = group*x_col_group + k
+  int x_col_group;
+  int stages;
+  // epilogue
+  void* out;             // bf16 output or fp32 partials
+  long out_ld;           // elements between consecutive b
+  long out_group;        // elements between consecutive groups
+  long out_split;        // fp32 partials: elements between K splits
+  // absorb epilogue (RoPE of q_pe into q_lat[:, h, d_c:])
+  const __nv_bfloat16* q_pe;
+  const int32_t* pos;
+  const float2* rope_cs;
+  int num_heads, d_c, d_r, max_position;
+  int* err;
+  uint32_t wait_limit;
+};
+
+template <bool kAMn, Epi kEpi>
+__global__ void __launch_bounds__(256, 2)
+    gemm_wt_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmX,
+                   const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = ptx::smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tiles = p.m_per_group / kM;
+  const int group = blockIdx.x / m_tiles;
+  const int m0 = (blockIdx.x % m_tiles) * kM;
+  const int split = blockIdx.y;
+  const int kc0 = static_cast<int>((static_cast<long>(split) * p.k_chunks) / p.k_split);
+  const int kc1 = static_cast<int>((static_cast<long>(split + 1) * p.k_chunks) / p.k_split);
+  const int nk = kc1 - kc0;
+
+  const int a_bytes = kM * kKc * 2;            // 16 KB
+  const int x_bytes = p.n * kKc * 2;           // n rows of 128 B
+  const int stage_bytes = a_bytes + x_bytes;   // multiple of 1024 (n % 8 == 0)
+  const uint32_t bars = sb + p.stages * stage_bytes;
+  auto full = [&](int s) { return bars + 8u * s; };
+  auto empty = [&](int s) { return bars + 8u * (p.stages + s); };
+  const uint32_t done = bars + 8u * (2 * p.stages);
+  const uint32_t drainb = done + 8u;
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + p.stages * stage_bytes +
+                                                                 8 * (2 * p.stages + 2));
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      ptx::mbar_init(full(s), 1);
+      ptx::mbar_init(empty(s), 1);
+    }
+    ptx::mbar_init(done, 1);
+    ptx::mbar_init(drainb, 1);
+    misc[1] = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  const uint32_t ncols = p.n <= 32 ? 32u : (p.n <= 64 ? 64u : (p.n <= 128 ? 128u : 256u));
+  if (warp == 1) {
+    ptx::tmem_alloc(sb + p.stages * stage_bytes + 8 * (2 * p.stages + 2), ncols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  auto fail = [&]() {
+    misc[1] = 1u;
+    report_error(p.err, MLA_ERR_TIMEOUT);
+  };
+  auto wait = [&](uint32_t b_, uint32_t par) -> bool {
+    if (misc[1]) return false;
+    const bool ok = ptx::mbar_wait<false>(b_, par, p.wait_limit, kWaitNs);
+    if (!ok) fail();
+    return ok;
+  };
+
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmX);
+    int issued = 0;
+    for (int i = 0; i < nk; ++i) {
+      const int s = i % p.stages;
+      if (!wait(empty(s), ((i / p.stages) & 1) ^ 1)) break;
+      const int k = (kc0 + i) * kKc;
+      const uint32_t dA = sb + s * stage_bytes, dX = dA + a_bytes;
+      ptx::mbar_arrive_expect_tx(full(s), stage_bytes);
+      if (kAMn) {
+        // two 64-wide boxes along M, 64 rows of K each
+        ptx::tma_load_2d(dA, &tmA, full(s), m0, group * p.a_row_group + k);
+        ptx::tma_load_2d(dA + kM * 64, &tmA, full(s), m0 + 64, group * p.a_row_group + k);
+      } else {
+        ptx::tma_load_2d(dA, &tmA, full(s), k, group * p.a_row_group + m0);
+      }
+      ptx::tma_load_2d(dX, &tmX, full(s), group * p.x_col_group + k, 0);
+      issued = i + 1;
+    }
+    for (int i = max(0, issued - p.stages); i < issued; ++i)
+      ptx::mbar_wait<false>(full(i % p.stages), (i / p.stages) & 1, 0xffffffffu, kWaitNs);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = ptx::idesc_bf16_f32(kM, p.n, kAMn, false);
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % p.stages;
+        if (!wait(full(s), (i / p.stages) & 1)) break;
+        ptx::tc_fence_after();
+        const uint32_t aB = sb + s * stage_bytes, xB = aB + a_bytes;
+#pragma unroll
+        for (int j = 0; j < kKc / 16; ++j) {
+          const uint64_t ad = kAMn ? ptx::sdesc_sw128(aB + j * 2048, 64 * 128, 1024)
+                                   : ptx::sdesc_sw128(aB + 32 * j, 16, 1024);
+          const uint64_t xd = ptx::sdesc_sw128(xB + 32 * j, 16, 1024);
+          ptx::umma_ss(tmem, ad, xd, idesc, (i > 0 || j > 0) ? 1u : 0u);
+        }
+        ptx::umma_commit(empty(s));
+      }
+      ptx::umma_commit(done);
+      ptx::umma_commit(drainb);
+      ptx::mbar_wait<false>(drainb, 0, 0xffffffffu, kWaitNs);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    const int q = warp & 3;
+    const int m = q * 32 + lane;                       // row of this thread in the tile
+    const uint32_t lb = static_cast<uint32_t>(q * 32) << 16;
+    if (kEpi == Epi::kAbsorb && (blockIdx.x % m_tiles) == 0 && split == 0) {
+      // RoPE(q_pe[b][h], pos[b]) -> q_lat[b][h][d_c:], pairs (i, i + d_r/2)
+      const int half = p.d_r / 2;
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+      for (int idx = m; idx < p.batch * half; idx += 128) {
+        const int b = idx / half, i = idx % half;
+        const int ps = p.pos[b];
+        if (ps < 0 || ps >= p.max_position) {
+          report_error(p.err, MLA_ERR_BAD_INDEX);
+          continue;
+        }
+        const float2 r = p.rope_cs[static_cast<long>(ps) * half + i];
+        const long qb = (static_cast<long>(b) * p.num_heads + group) * p.d_r;
+        const float x1 = __bfloat162float(p.q_pe[qb + i]), x2 = __bfloat162float(p.q_pe[qb + half + i]);
+        const long ob = b * p.out_ld + group * p.out_group + p.d_c;
+        out[ob + i] = __float2bfloat16_rn(x1 * r.x - x2 * r.y);
+        out[ob + half + i] = __float2bfloat16_rn(x2 * r.x + x1 * r.y);
+      }
+    }
+    bool ok = wait(done, 0);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && nk > 0) {
+      ptx::tc_fence_after();
+      for (int c0 = 0; c0 < p.n; c0 += 32) {
+        uint32_t v[32];
+        ptx::tmem_ld32(tmem + lb + c0, v);
+        ptx::tmem_wait_ld();
+        if (kEpi == Epi::kPartialF32) {
+          float* out = reinterpret_cast<float*>(p.out) + split * p.out_split + group * p.out_group + m0 + m;
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c0 + e < p.batch) out[(c0 + e) * p.out_ld] = __uint_as_float(v[e]);
+        } else {
+          __nv_bfloat16* out =
+              reinterpret_cast<__nv_bfloat16*>(p.out) + group * p.out_group + m0 + m;
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c0 + e < p.batch) out[(c0 + e) * p.out_ld] = __float2bfloat16_rn(__uint_as_float(v[e]));
+        }
+      }
+      ptx::tc_fence_before();
+    }
+  }
+  __syncwarp();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, ncols);
+  }
+}
+
+// y[b][m] = sum_s partial[s][b][m] in bf16.
+__global__ void __launch_bounds__(256) reduce_splits_kernel(const float* __restrict__ part,
+                                                            __nv_bfloat16* __restrict__ y,
+                                                            int splits, long count) {
+  for (long i = blockIdx.x * 256L + threadIdx.x; i < count; i += gridDim.x * 256L) {
+    float s = 0.f;
+    for (int k = 0; k < splits; ++k) s += part[k * count + i];
+    y[i] = __float2bfloat16_rn(s);
+  }
+}
+
+}  // namespace gemm
+}  // namespace mla

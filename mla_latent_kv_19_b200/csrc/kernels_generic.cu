@@ -353,6 +353,7 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(DecodeArgs 
   }
   __syncthreads();
   const long part = (static_cast<long>(b) * a.num_splits + split) * a.num_heads;
+  const long obase = (static_cast<long>(b) * a.num_splits + split) * a.d_c;   // o_part[b][s][c][h]
 #pragma unroll
   for (int jc = 0; jc < kGenColsPerThread; ++jc) {
     const int c = tid + jc * kGenThreads;
@@ -361,7 +362,7 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(DecodeArgs 
       for (int g = 0; g < kGenHeads; ++g) {
         if (g < nh) {
           const float l = ps[g];
-          a.o_part[(part + h0 + g) * a.d_c + c] = l > 0.f ? acc[g][jc] / l : 0.f;
+          a.o_part[(obase + c) * a.num_heads + h0 + g] = l > 0.f ? acc[g][jc] / l : 0.f;
         }
       }
     }
@@ -402,53 +403,62 @@ cudaError_t launch_decode_generic(const DecodeArgs& a, int act_dtype, int cache_
 // split merge by log-sum-exp
 // ---------------------------------------------------------------------------
 
+// One CTA per (sequence b, chunk of 32 latent columns); thread = head.  Reads
+// o_part[b][s][c][h] (coalesced over heads), merges the splits with weights
+// exp(lse_s - lse), transposes through shared memory and writes o_lat[b][h][c]
+// rows of 32 contiguous columns.
+constexpr int kCombCols = 32;
+
 template <typename T>
 __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
-  extern __shared__ float w_s[];  // [num_splits]
-  __shared__ float inv_z_s, lse_s;
-  const int b = blockIdx.x, h = blockIdx.y;
-  const int S = a.num_splits;
-  const long part0 = static_cast<long>(b) * S * a.num_heads + h;
-  if (threadIdx.x < 32) {
+  extern __shared__ float cw[];               // [num_splits][H] weights
+  __shared__ float tile[kCombCols][129];      // [c][h], padded
+  const int b = blockIdx.x, c0 = blockIdx.y * kCombCols;
+  const int S = a.num_splits, H = a.num_heads;
+  const int h = threadIdx.x;                  // blockDim.x == 128 >= H
+  float inv_z = 0.f;
+  if (h < H) {
+    const float* lp = a.lse_part + static_cast<long>(b) * S * H + h;
     float m = -INFINITY;
-    for (int s = threadIdx.x; s < S; s += 32) m = fmaxf(m, a.lse_part[part0 + static_cast<long>(s) * a.num_heads]);
-    m = warp_max(m);
+    for (int s = 0; s < S; ++s) m = fmaxf(m, lp[static_cast<long>(s) * H]);
     float z = 0.f;
-    for (int s = threadIdx.x; s < S; s += 32) {
-      const float l = a.lse_part[part0 + static_cast<long>(s) * a.num_heads];
-      const float w = (m == -INFINITY) ? 0.f : __expf(l - m);
-      w_s[s] = w;
+    for (int s = 0; s < S; ++s) {
+      const float w = (m == -INFINITY) ? 0.f : __expf(lp[static_cast<long>(s) * H] - m);
+      cw[s * H + h] = w;
       z += w;
     }
-    z = warp_sum(z);
-    if (threadIdx.x == 0) {
-      inv_z_s = z > 0.f ? 1.f / z : 0.f;
-      lse_s = z > 0.f ? m + __logf(z) : -INFINITY;
+    inv_z = z > 0.f ? 1.f / z : 0.f;
+    if (blockIdx.y == 0 && a.lse != nullptr)
+      a.lse[static_cast<long>(b) * H + h] = z > 0.f ? m + __logf(z) : -INFINITY;
+    const float* op = a.o_part + static_cast<long>(b) * S * a.d_c * H + h;
+    for (int c = 0; c < kCombCols && c0 + c < a.d_c; ++c) {
+      float o = 0.f;
+      for (int s = 0; s < S; ++s) {
+        const float w = cw[s * H + h];
+        if (w != 0.f) o += w * op[(static_cast<long>(s) * a.d_c + c0 + c) * H];
+      }
+      tile[c][h] = o * inv_z;
     }
   }
   __syncthreads();
-  const float inv_z = inv_z_s;
-  T* out = reinterpret_cast<T*>(a.o_lat) + (static_cast<long>(b) * a.num_heads + h) * a.d_c;
-  for (int c = threadIdx.x; c < a.d_c; c += blockDim.x) {
-    float o = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float w = w_s[s];
-      if (w != 0.f) o += w * a.o_part[(part0 + static_cast<long>(s) * a.num_heads) * a.d_c + c];
-    }
-    out[c] = cvt_out<T>(o * inv_z);
-  }
-  if (threadIdx.x == 0 && a.lse != nullptr) a.lse[static_cast<long>(b) * a.num_heads + h] = lse_s;
+  // o_lat[b][hh][c0 + cc]: a warp writes one head row of 32 columns per step
+  T* out = reinterpret_cast<T*>(a.o_lat) + static_cast<long>(b) * H * a.d_c;
+  const int cc = threadIdx.x & 31;
+  for (int hh = threadIdx.x >> 5; hh < H; hh += 4)
+    if (c0 + cc < a.d_c) out[static_cast<long>(hh) * a.d_c + c0 + cc] = cvt_out<T>(tile[cc][hh]);
 }
 
 cudaError_t launch_combine(const CombineArgs& a, int act_dtype, cudaStream_t s) {
   if (a.batch == 0) return cudaSuccess;
-  dim3 grid(a.batch, a.num_heads);
-  size_t smem = sizeof(float) * a.num_splits;
-  if (act_dtype == MLA_FP32) {
-    combine_kernel<float><<<grid, 128, smem, s>>>(a);
-  } else {
-    combine_kernel<__nv_bfloat16><<<grid, 128, smem, s>>>(a);
+  if (a.num_heads > 128) return cudaErrorInvalidValue;
+  dim3 grid(a.batch, (a.d_c + kCombCols - 1) / kCombCols);
+  const size_t smem = sizeof(float) * a.num_splits * a.num_heads;
+  void (*k)(CombineArgs) = act_dtype == MLA_FP32 ? combine_kernel<float> : combine_kernel<__nv_bfloat16>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
   }
+  k<<<grid, 128, smem, s>>>(a);
   note_launches(1);
   return cudaGetLastError();
 }

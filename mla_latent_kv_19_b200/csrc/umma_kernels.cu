@@ -1,9 +1,11 @@
 // tcgen05 / TMEM / TMA kernels of libmla (sm_100a) and their launchers.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "decode_umma.cuh"
+#include "gemm_umma.cuh"
 #include "umma_kernels.h"
 
 namespace mla {
@@ -22,6 +24,25 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   });
   return fn;
+}
+
+// Rows of `chunks` x 64 bf16 columns read as a 3-D tensor (64 columns, rows,
+// column chunk), so that one box of box_rows x chunks lands in shared memory
+// chunk-major: [chunk][row][128 bytes], 128-byte swizzled -- the UMMA K-major
+// (and, for V, MN-major) operand layout.
+cudaError_t make_map_rows_chunked(CUtensorMap* map, const void* base, uint64_t rows,
+                                  uint64_t row_bytes, uint32_t chunks, uint32_t box_rows,
+                                  uint32_t box_chunks) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {64, rows, chunks};
+  const cuuint64_t strides[2] = {row_bytes, 128};
+  const cuuint32_t box[3] = {64, box_rows, box_chunks};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 // 2-D bf16 tensor map, 128-byte swizzle, box = box_cols x box_rows.
@@ -53,9 +74,16 @@ bool umma_decode_supported(const mla_ctx* h) {
 }
 
 cudaError_t launch_decode_umma(const mla_ctx* h, const DecodeArgs& a, cudaStream_t s) {
-  CUtensorMap map;
-  cudaError_t e = make_map_bf16(&map, a.cache, dec::kD, static_cast<uint64_t>(a.num_blocks) * dec::kTok,
-                                dec::kD * 2, 64, 64);
+  CUtensorMap kmap, vmap, qmap;
+  const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * dec::kTok;
+  cudaError_t e = make_map_rows_chunked(&kmap, a.cache, rows, dec::kD * 2, dec::kKBoxes, dec::kTok,
+                                        dec::kKBoxes);
+  if (e != cudaSuccess) return e;
+  e = make_map_rows_chunked(&vmap, a.cache, rows, dec::kD * 2, dec::kKBoxes, dec::kTok, dec::kVBoxes);
+  if (e != cudaSuccess) return e;
+  // absorbed queries as [B*H rows][576 columns], half of a sequence's heads per box
+  e = make_map_rows_chunked(&qmap, a.q_lat, static_cast<uint64_t>(a.batch) * dec::kH, dec::kD * 2,
+                            dec::kKBoxes, 64, dec::kKBoxes);
   if (e != cudaSuccess) return e;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
@@ -66,23 +94,156 @@ cudaError_t launch_decode_umma(const mla_ctx* h, const DecodeArgs& a, cudaStream
   if (attr_err != cudaSuccess) return attr_err;
   const long ctas = 2L * a.batch * a.num_splits;
   if (ctas > 0x7fffffffL) return cudaErrorInvalidValue;
-  dec::decode_umma_kernel<<<dim3(static_cast<unsigned>(ctas)), 256, dec::kSmemBytes, s>>>(map, a);
+  dec::decode_umma_kernel<<<dim3(static_cast<unsigned>(ctas)), 256, dec::kSmemBytes, s>>>(kmap, vmap, qmap, a);
   note_launches(1);
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// absorb and output projection: not yet on tensor cores
+// projections: weight-streaming tcgen05 GEMM
 // ---------------------------------------------------------------------------
 
-bool umma_absorb_supported(const mla_ctx*, int) { return false; }
-cudaError_t launch_absorb_umma(const mla_ctx*, const AbsorbArgs&, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int kOProjSplits = 7;      // K split of W_O: 40 row tiles x 7 = 280 CTAs, two per SM
+constexpr int kGemmStages = 5;
+
+int padded_n(int batch) { return (batch + 15) / 16 * 16; }
+
+size_t gemm_smem_bytes(int n, int stages) {
+  return static_cast<size_t>(stages) * (gemm::kM * gemm::kKc * 2 + n * gemm::kKc * 2) +
+         8 * (2 * stages + 2) + 16 + 1024;
 }
-bool umma_out_proj_supported(const mla_ctx*, int) { return false; }
-size_t umma_out_proj_extra_workspace(const mla_ctx*, int) { return 0; }
-cudaError_t launch_out_proj_umma(const mla_ctx*, const OutProjArgs&, void*, cudaStream_t) {
-  return cudaErrorNotSupported;
+
+template <bool kAMn, gemm::Epi kEpi>
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tx, const gemm::Params& p,
+                        dim3 grid, cudaStream_t s) {
+  const size_t smem = gemm_smem_bytes(p.n, p.stages);
+  cudaError_t e = cudaFuncSetAttribute(gemm::gemm_wt_kernel<kAMn, kEpi>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  gemm::gemm_wt_kernel<kAMn, kEpi><<<grid, 256, smem, s>>>(ta, tx, p);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+bool v2_bf16(const mla_ctx* h) {
+  const mla_config_t& c = h->cfg;
+  return h->cc_major == 10 && c.act_dtype == MLA_BF16 && c.num_heads == 128 && c.d_c == 512 &&
+         c.d_r == 64 && c.d_nope == 128 && c.d_v == 128 && c.d_model % 128 == 0 &&
+         encode_fn() != nullptr;
+}
+
+}  // namespace
+
+bool umma_absorb_supported(const mla_ctx* h, int batch) {
+  return v2_bf16(h) && batch >= 1 && batch <= 256;
+}
+
+cudaError_t launch_absorb_umma(const mla_ctx* h, const AbsorbArgs& a, cudaStream_t s) {
+  const int H = a.num_heads, n = padded_n(a.batch);
+  CUtensorMap ta, tx;
+  // W_UK viewed as [H*d_nope rows (k)][d_c cols (c)], read MN-major in 64x64 boxes
+  cudaError_t e = make_map_bf16(&ta, a.w_uk, a.d_c, static_cast<uint64_t>(H) * a.d_nope, a.d_c * 2, 64, 64);
+  if (e != cudaSuccess) return e;
+  // q_nope viewed as [B rows][H*d_nope cols]
+  e = make_map_bf16(&tx, a.q_nope, static_cast<uint64_t>(H) * a.d_nope, a.batch,
+                    static_cast<uint64_t>(H) * a.d_nope * 2, 64, n);
+  if (e != cudaSuccess) return e;
+  gemm::Params p{};
+  p.n = n;
+  p.batch = a.batch;
+  p.k_chunks = a.d_nope / gemm::kKc;
+  p.k_split = 1;
+  p.m_per_group = a.d_c;
+  p.a_row_group = a.d_nope;
+  p.x_col_group = a.d_nope;
+  p.stages = 2;
+  p.out = a.q_lat;
+  p.out_ld = static_cast<long>(H) * (a.d_c + a.d_r);
+  p.out_group = a.d_c + a.d_r;
+  p.q_pe = static_cast<const __nv_bfloat16*>(a.q_pe);
+  p.pos = a.pos;
+  p.rope_cs = a.rope_cs;
+  p.num_heads = H;
+  p.d_c = a.d_c;
+  p.d_r = a.d_r;
+  p.max_position = a.max_position;
+  p.err = a.err;
+  p.wait_limit = h->wait_limit;
+  return launch_gemm<true, gemm::Epi::kAbsorb>(ta, tx, p, dim3(H * (a.d_c / gemm::kM), 1), s);
+}
+
+bool umma_out_proj_supported(const mla_ctx* h, int batch) {
+  return v2_bf16(h) && batch >= 1 && batch <= 256;
+}
+
+size_t umma_out_proj_extra_workspace(const mla_ctx* h, int batch) {
+  if (!umma_out_proj_supported(h, batch)) return 0;
+  return static_cast<size_t>(kOProjSplits) * batch * h->cfg.d_model * sizeof(float) + 256;
+}
+
+cudaError_t launch_out_proj_umma(const mla_ctx* h, const OutProjArgs& a, void* extra,
+                                 cudaStream_t s) {
+  const int H = a.num_heads, n = padded_n(a.batch);
+  const long kdim = static_cast<long>(H) * a.d_v;
+  // o[b][h][v] = W_UV[h] o_lat[b][h]
+  {
+    CUtensorMap ta, tx;
+    cudaError_t e = make_map_bf16(&ta, a.w_uv, a.d_c, static_cast<uint64_t>(H) * a.d_v, a.d_c * 2, 64, 128);
+    if (e != cudaSuccess) return e;
+    e = make_map_bf16(&tx, a.o_lat, static_cast<uint64_t>(H) * a.d_c, a.batch,
+                      static_cast<uint64_t>(H) * a.d_c * 2, 64, n);
+    if (e != cudaSuccess) return e;
+    gemm::Params p{};
+    p.n = n;
+    p.batch = a.batch;
+    p.k_chunks = a.d_c / gemm::kKc;
+    p.k_split = 1;
+    p.m_per_group = a.d_v;
+    p.a_row_group = a.d_v;
+    p.x_col_group = a.d_c;
+    p.stages = 4;
+    p.out = a.o;
+    p.out_ld = kdim;
+    p.out_group = a.d_v;
+    p.err = h->err;
+    p.wait_limit = h->wait_limit;
+    e = launch_gemm<false, gemm::Epi::kStoreBf16T>(ta, tx, p, dim3(H, 1), s);
+    if (e != cudaSuccess) return e;
+  }
+  // partial[s][b][m] = sum over this split's K of W_O[m][k] o[b][k]
+  float* part = static_cast<float*>(extra);
+  {
+    CUtensorMap ta, tx;
+    cudaError_t e = make_map_bf16(&ta, a.w_o, kdim, a.d_model, kdim * 2, 64, 128);
+    if (e != cudaSuccess) return e;
+    e = make_map_bf16(&tx, a.o, kdim, a.batch, kdim * 2, 64, n);
+    if (e != cudaSuccess) return e;
+    gemm::Params p{};
+    p.n = n;
+    p.batch = a.batch;
+    p.k_chunks = static_cast<int>(kdim / gemm::kKc);
+    p.k_split = kOProjSplits;
+    p.m_per_group = a.d_model;
+    p.a_row_group = 0;
+    p.x_col_group = 0;
+    p.stages = kGemmStages;
+    p.out = part;
+    p.out_ld = a.d_model;
+    p.out_group = 0;
+    p.out_split = static_cast<long>(a.batch) * a.d_model;
+    p.err = h->err;
+    p.wait_limit = h->wait_limit;
+    e = launch_gemm<false, gemm::Epi::kPartialF32>(ta, tx, p, dim3(a.d_model / gemm::kM, kOProjSplits), s);
+    if (e != cudaSuccess) return e;
+  }
+  const long count = static_cast<long>(a.batch) * a.d_model;
+  gemm::reduce_splits_kernel<<<static_cast<unsigned>(std::min<long>((count + 255) / 256, 1184)), 256, 0, s>>>(
+      part, static_cast<__nv_bfloat16*>(a.y), kOProjSplits, count);
+  note_launches(1);
+  return cudaGetLastError();
 }
 
 }  // namespace mla

@@ -136,7 +136,8 @@ def test_combine_against_oracle_merge():
     nbytes = mla_decode_workspace_bytes(h, B, S, 64 * S)
     ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
     n_o = B * S * H * dc * 4
-    ws[:n_o].view(torch.float32).copy_(torch.from_numpy(o.reshape(-1)))
+    # workspace layout o_part[b][s][c][h]
+    ws[:n_o].view(torch.float32).copy_(torch.from_numpy(np.ascontiguousarray(o.transpose(0, 1, 3, 2)).reshape(-1)))
     off = (n_o + 255) // 256 * 256
     ws[off:off + B * S * H * 4].view(torch.float32).copy_(torch.from_numpy(lse.reshape(-1)))
     o_lat = torch.empty(B, H, dc, dtype=torch.bfloat16, device="cuda")
