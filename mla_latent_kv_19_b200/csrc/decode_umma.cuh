@@ -88,7 +88,9 @@ enum Bar {
   kDrain = kFin + 1, kNumBars = kDrain + 1
 };
 constexpr int kOffBar = kRegionEnd;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;       // [0] tmem base, [1] abort, [2] corr tile
+// misc words: [0] tmem base, [1] abort, [2] corr tile, [3] P messages CTA 0 sent
+// (written by CTA 0 into CTA 1), [4] messages CTA 1 consumed, [5] messages it armed
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;       // + slack for the 1024-byte alignment
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -207,6 +209,9 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
     ptx::mbar_init(bar(kDrain), 1);
     misc[1] = 0u;
     misc[2] = 0u;
+    misc[3] = 0u;
+    misc[4] = 0u;
+    misc[5] = 0u;
     ptx::fence_mbar_init_cluster();
   }
   __syncwarp();
@@ -316,6 +321,7 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
       const uint32_t rFin = ptx::mapa(bar(kFin), 1);
       const float sl2 = a.scale * kLog2e;
       float m_used = -INFINITY, l = 0.f;
+      uint32_t sent = 0;
 #pragma unroll 1
       for (int t = 0; t < sp.ntiles && ok; ++t) {
         const int i = t & 1;
@@ -370,9 +376,11 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
         ptx::mbar_arrive(bar(kStg + i));
         if (r == 0) {
           // every row of the message is written: ship it to CTA 1 in one bulk copy
-          if (wait_local(bar(kStg + i), (t >> 1) & 1))
+          if (wait_local(bar(kStg + i), (t >> 1) & 1)) {
             ptx::bulk_copy_to_peer(rP + (t % kPBufs) * kPBufStride, sb + kOffRing + slot * kSlotBytes,
                                    kPMsgBytes, rPFull + 8u * (t % kPBufs));
+            ++sent;
+          }
         }
       }
       // this split's log-sum-exp (natural log) and the normaliser for CTA 1
@@ -380,6 +388,7 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
       a.lse_part[row] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
       ptx::st_cluster_u32(rL + r * 4, __float_as_uint(l));
       ptx::mbar_arrive_remote(rFin);
+      if (r == 0) ptx::st_cluster_u32(ptx::mapa(sb + kOffMisc + 12, 1), sent);
     }
   } else {
     // =========================== CTA 1: values ===========================
@@ -408,10 +417,14 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
 #pragma unroll 1
       for (int t = 0; t < sp.ntiles; ++t) {
         const int st = t & 1, pbi = t % kPBufs;
-        if (lane == 0) ptx::mbar_arrive_expect_tx(bar(kPFull + pbi), kPMsgBytes);
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(bar(kPFull + pbi), kPMsgBytes);
+          misc[5] = static_cast<uint32_t>(t + 1);
+        }
         bool ok = wait_local(bar(kVFull + st), (t >> 1) & 1);
         ok = ok && wait_remote(bar(kPFull + pbi), (t / kPBufs) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
+        if (lane == 0) misc[4] = static_cast<uint32_t>(t + 1);
         const int valid = valid_tokens(sp, page_at(a, sp, table, t), t);
         if (valid < kTok) {
           // rows past the sequence end: zero them so that P = 0 meets finite V
@@ -536,7 +549,19 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
 
   __syncwarp();
   __syncthreads();
-  ptx::cluster_sync();       // no remote access to this CTA's shared memory after this point
+  ptx::cluster_sync();       // CTA 1 now sees how many P messages CTA 0 sent
+  if (rank == 1 && threadIdx.x == 0) {
+    // after a wait gave up, messages may still be landing: arm and await each one
+    // not consumed yet (in order, so that phase parities stay in step)
+    const uint32_t sent = misc[3], armed = misc[5];
+    for (uint32_t t = misc[4]; t < sent; ++t) {
+      if (t >= armed) ptx::mbar_arrive_expect_tx(bar(kPFull + t % kPBufs), kPMsgBytes);
+      drain(bar(kPFull + t % kPBufs), (t / kPBufs) & 1);
+    }
+  }
+  __syncwarp();
+  __syncthreads();
+  ptx::cluster_sync();       // no copy in flight and no remote access after this point
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);

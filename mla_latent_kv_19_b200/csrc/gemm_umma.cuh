@@ -3,8 +3,8 @@
 //
 //   D[m][b] = sum_k A[m][k] * X[b][k]
 //
-// with the weight as the M operand (128 rows per CTA, "swap-AB": the batch is
-// the N dimension, 16 <= N <= 256) and fp32 accumulation in TMEM.  Uses:
+// with the weight as the M operand (128 rows per tile, "swap-AB": the batch
+// is the N dimension, 16 <= N <= 256) and fp32 accumulation in TMEM.  Uses:
 //   * W_O   (V2 page section 2.3, W_UV absorbed into W_O; applied as W_O after
 //            W_UV):  A = W_O [5120][16384] K-major, X = o [B][16384];
 //            K split over CTAs, fp32 partials reduced by a second kernel.
@@ -13,9 +13,12 @@
 //            i.e. W_UK[h] [128][512] read MN-major, X = q_nope[:, h, :];
 //            the epilogue also applies RoPE to q_pe (section 2.2).
 //
-// The kernel is HBM-bound on the weight stream (2 flops per weight byte per
-// token of the batch); a TMA ring of (A, X) chunks of 64 along K keeps enough
-// bytes in flight per SM, one thread issues the UMMAs, four warps drain TMEM.
+// HBM-bound on the weight stream (2 flops per weight byte per token of the
+// batch).  Each pipeline stage is ONE 3-D TMA request for A (kcs chunks of 64
+// along K, landing chunk-major in the 128-byte-swizzled UMMA layout) and one
+// for X, so a stage moves 16*kcs KB of weights with two requests; a CTA may
+// own several consecutive M tiles of one group, each accumulating in its own
+// TMEM columns.  One thread issues the UMMAs, four warps drain TMEM.
 #pragma once
 
 #include "device_common.cuh"
@@ -24,8 +27,8 @@
 namespace mla {
 namespace gemm {
 
-constexpr int kM = 128;          // weight rows per CTA
-constexpr int kKc = 64;          // K per pipeline stage (one 128-byte swizzle row of bf16)
+constexpr int kM = 128;          // weight rows per tile
+constexpr int kKc = 64;          // K per chunk (one 128-byte swizzle row of bf16)
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 enum class Epi : int { kStoreBf16T = 0, kPartialF32 = 1, kAbsorb = 2 };
@@ -36,10 +39,12 @@ struct Params {
   int k_chunks;          // K / 64 per group
   int k_split;           // CTAs along K (gridDim.y)
   int m_per_group;       // weight rows of one group (head), multiple of 128
-  // A coordinates: K-major: row = group*a_row_group + m, col = k
-  //                MN-major: row = group*a_row_group + k, col = m
+  int mt_per_cta;        // M tiles of one group handled by one CTA
+  int kcs;               // K chunks per pipeline stage (box depth)
+  // A coordinates: K-major: (elem, row = group*a_row_group + m, chunk = k/64)
+  //                MN-major: (elem, row = group*a_row_group + k, chunk = m/64)
   int a_row_group;
-  // X coordinates: row = b, col = group*x_col_group + k
+  // X coordinates: (elem, row = b, chunk = (group*x_col_group + k)/64)
   int x_col_group;
   int stages;
   // epilogue
@@ -57,7 +62,7 @@ struct Params {
 };
 
 template <bool kAMn, Epi kEpi>
-__global__ void __launch_bounds__(256, 2)
+__global__ void __launch_bounds__(256, 1)
     gemm_wt_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmX,
                    const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -66,16 +71,18 @@ __global__ void __launch_bounds__(256, 2)
   const uint32_t sb = ptx::smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m_tiles = p.m_per_group / kM;
-  const int group = blockIdx.x / m_tiles;
-  const int m0 = (blockIdx.x % m_tiles) * kM;
+  const int cta_per_group = m_tiles / p.mt_per_cta;
+  const int group = blockIdx.x / cta_per_group;
+  const int mt0 = (blockIdx.x % cta_per_group) * p.mt_per_cta;
   const int split = blockIdx.y;
   const int kc0 = static_cast<int>((static_cast<long>(split) * p.k_chunks) / p.k_split);
   const int kc1 = static_cast<int>((static_cast<long>(split + 1) * p.k_chunks) / p.k_split);
-  const int nk = kc1 - kc0;
+  const int nst_k = (kc1 - kc0 + p.kcs - 1) / p.kcs;     // stages per M tile
+  const int nst = nst_k * p.mt_per_cta;
 
-  const int a_bytes = kM * kKc * 2;            // 16 KB
-  const int x_bytes = p.n * kKc * 2;           // n rows of 128 B
-  const int stage_bytes = a_bytes + x_bytes;   // multiple of 1024 (n % 8 == 0)
+  const int a_bytes = kM * kKc * 2 * p.kcs;              // 16 KB per chunk
+  const int x_bytes = p.n * kKc * 2 * p.kcs;             // n rows of 128 B per chunk
+  const int stage_bytes = a_bytes + x_bytes;             // multiple of 1024 (n % 8 == 0)
   const uint32_t bars = sb + p.stages * stage_bytes;
   auto full = [&](int s) { return bars + 8u * s; };
   auto empty = [&](int s) { return bars + 8u * (p.stages + s); };
@@ -83,6 +90,10 @@ __global__ void __launch_bounds__(256, 2)
   const uint32_t drainb = done + 8u;
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + p.stages * stage_bytes +
                                                                  8 * (2 * p.stages + 2));
+  // TMEM: one block of ncpt columns per M tile
+  const uint32_t ncpt = p.n <= 32 ? 32u : (p.n <= 64 ? 64u : (p.n <= 128 ? 128u : 256u));
+  uint32_t ncols = 32;
+  while (ncols < ncpt * p.mt_per_cta) ncols <<= 1;
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
       ptx::mbar_init(full(s), 1);
@@ -94,7 +105,6 @@ __global__ void __launch_bounds__(256, 2)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncwarp();
-  const uint32_t ncols = p.n <= 32 ? 32u : (p.n <= 64 ? 64u : (p.n <= 128 ? 128u : 256u));
   if (warp == 1) {
     ptx::tmem_alloc(sb + p.stages * stage_bytes + 8 * (2 * p.stages + 2), ncols);
     ptx::tmem_relinquish();
@@ -115,42 +125,51 @@ __global__ void __launch_bounds__(256, 2)
     return ok;
   };
 
-  if (warp == 0 && lane == 0) {
-    ptx::prefetch_tmap(&tmA);
-    ptx::prefetch_tmap(&tmX);
-    int issued = 0;
-    for (int i = 0; i < nk; ++i) {
-      const int s = i % p.stages;
-      if (!wait(empty(s), ((i / p.stages) & 1) ^ 1)) break;
-      const int k = (kc0 + i) * kKc;
-      const uint32_t dA = sb + s * stage_bytes, dX = dA + a_bytes;
-      ptx::mbar_arrive_expect_tx(full(s), stage_bytes);
-      if (kAMn) {
-        // two 64-wide boxes along M, 64 rows of K each
-        ptx::tma_load_2d(dA, &tmA, full(s), m0, group * p.a_row_group + k);
-        ptx::tma_load_2d(dA + kM * 64, &tmA, full(s), m0 + 64, group * p.a_row_group + k);
-      } else {
-        ptx::tma_load_2d(dA, &tmA, full(s), k, group * p.a_row_group + m0);
+  if (warp == 0) {
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmA);
+      ptx::prefetch_tmap(&tmX);
+      int issued = 0;
+      for (int i = 0; i < nst; ++i) {
+        const int s = i % p.stages;
+        if (!wait(empty(s), ((i / p.stages) & 1) ^ 1)) break;
+        const int mt = mt0 + i / nst_k;
+        const int kc = kc0 + (i % nst_k) * p.kcs;
+        const uint32_t dA = sb + s * stage_bytes, dX = dA + a_bytes;
+        ptx::mbar_arrive_expect_tx(full(s), stage_bytes);
+        if (kAMn) {
+          // rows = K (kcs*64 of them), chunks = two 64-wide slices of this M tile
+          ptx::tma_load_3d(dA, &tmA, full(s), 0, group * p.a_row_group + kc * kKc, mt * 2);
+        } else {
+          ptx::tma_load_3d(dA, &tmA, full(s), 0, group * p.a_row_group + mt * kM, kc);
+        }
+        ptx::tma_load_3d(dX, &tmX, full(s), 0, 0, (group * p.x_col_group) / kKc + kc);
+        issued = i + 1;
       }
-      ptx::tma_load_2d(dX, &tmX, full(s), group * p.x_col_group + k, 0);
-      issued = i + 1;
+      for (int i = max(0, issued - p.stages); i < issued; ++i)
+        ptx::mbar_wait<false>(full(i % p.stages), (i / p.stages) & 1, 0xffffffffu, kWaitNs);
     }
-    for (int i = max(0, issued - p.stages); i < issued; ++i)
-      ptx::mbar_wait<false>(full(i % p.stages), (i / p.stages) & 1, 0xffffffffu, kWaitNs);
+    __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = ptx::idesc_bf16_f32(kM, p.n, kAMn, false);
-      for (int i = 0; i < nk; ++i) {
+      for (int i = 0; i < nst; ++i) {
         const int s = i % p.stages;
         if (!wait(full(s), (i / p.stages) & 1)) break;
         ptx::tc_fence_after();
         const uint32_t aB = sb + s * stage_bytes, xB = aB + a_bytes;
+        const uint32_t d = tmem + ncpt * static_cast<uint32_t>(i / nst_k);
+        const int kin = i % nst_k;
+        const int nkc = min(p.kcs, kc1 - (kc0 + kin * p.kcs));   // chunks of this stage in range
+        for (int c = 0; c < nkc; ++c) {
 #pragma unroll
-        for (int j = 0; j < kKc / 16; ++j) {
-          const uint64_t ad = kAMn ? ptx::sdesc_sw128(aB + j * 2048, 64 * 128, 1024)
-                                   : ptx::sdesc_sw128(aB + 32 * j, 16, 1024);
-          const uint64_t xd = ptx::sdesc_sw128(xB + 32 * j, 16, 1024);
-          ptx::umma_ss(tmem, ad, xd, idesc, (i > 0 || j > 0) ? 1u : 0u);
+          for (int j = 0; j < kKc / 16; ++j) {
+            const uint64_t ad = kAMn
+                ? ptx::sdesc_sw128(aB + (c * kKc + 16 * j) * 128, kKc * p.kcs * 128, 1024)
+                : ptx::sdesc_sw128(aB + c * (kM * 128) + 32 * j, 16, 1024);
+            const uint64_t xd = ptx::sdesc_sw128(xB + c * (p.n * 128) + 32 * j, 16, 1024);
+            ptx::umma_ss(d, ad, xd, idesc, (kin > 0 || c > 0 || j > 0) ? 1u : 0u);
+          }
         }
         ptx::umma_commit(empty(s));
       }
@@ -161,9 +180,9 @@ __global__ void __launch_bounds__(256, 2)
     __syncwarp();
   } else if (warp >= 4) {
     const int q = warp & 3;
-    const int m = q * 32 + lane;                       // row of this thread in the tile
+    const int m = q * 32 + lane;                       // row of this thread in a tile
     const uint32_t lb = static_cast<uint32_t>(q * 32) << 16;
-    if (kEpi == Epi::kAbsorb && (blockIdx.x % m_tiles) == 0 && split == 0) {
+    if (kEpi == Epi::kAbsorb && mt0 == 0 && split == 0) {
       // RoPE(q_pe[b][h], pos[b]) -> q_lat[b][h][d_c:], pairs (i, i + d_r/2)
       const int half = p.d_r / 2;
       __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
@@ -184,23 +203,26 @@ __global__ void __launch_bounds__(256, 2)
     }
     bool ok = wait(done, 0);
     ok = __all_sync(0xffffffffu, ok);
-    if (ok && nk > 0) {
+    if (ok && nst > 0) {
       ptx::tc_fence_after();
-      for (int c0 = 0; c0 < p.n; c0 += 32) {
-        uint32_t v[32];
-        ptx::tmem_ld32(tmem + lb + c0, v);
-        ptx::tmem_wait_ld();
-        if (kEpi == Epi::kPartialF32) {
-          float* out = reinterpret_cast<float*>(p.out) + split * p.out_split + group * p.out_group + m0 + m;
+      for (int t = 0; t < p.mt_per_cta; ++t) {
+        const int m0 = (mt0 + t) * kM;
+        for (int c0 = 0; c0 < p.n; c0 += 32) {
+          uint32_t v[32];
+          ptx::tmem_ld32(tmem + lb + ncpt * t + c0, v);
+          ptx::tmem_wait_ld();
+          if (kEpi == Epi::kPartialF32) {
+            float* out = reinterpret_cast<float*>(p.out) + split * p.out_split + group * p.out_group + m0 + m;
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c0 + e < p.batch) out[(c0 + e) * p.out_ld] = __uint_as_float(v[e]);
-        } else {
-          __nv_bfloat16* out =
-              reinterpret_cast<__nv_bfloat16*>(p.out) + group * p.out_group + m0 + m;
+            for (int e = 0; e < 32; ++e)
+              if (c0 + e < p.batch) out[(c0 + e) * p.out_ld] = __uint_as_float(v[e]);
+          } else {
+            __nv_bfloat16* out =
+                reinterpret_cast<__nv_bfloat16*>(p.out) + group * p.out_group + m0 + m;
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c0 + e < p.batch) out[(c0 + e) * p.out_ld] = __float2bfloat16_rn(__uint_as_float(v[e]));
+            for (int e = 0; e < 32; ++e)
+              if (c0 + e < p.batch) out[(c0 + e) * p.out_ld] = __float2bfloat16_rn(__uint_as_float(v[e]));
+          }
         }
       }
       ptx::tc_fence_before();

@@ -431,14 +431,19 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
     if (blockIdx.y == 0 && a.lse != nullptr)
       a.lse[static_cast<long>(b) * H + h] = z > 0.f ? m + __logf(z) : -INFINITY;
     const float* op = a.o_part + static_cast<long>(b) * S * a.d_c * H + h;
-    for (int c = 0; c < kCombCols && c0 + c < a.d_c; ++c) {
-      float o = 0.f;
-      for (int s = 0; s < S; ++s) {
-        const float w = cw[s * H + h];
-        if (w != 0.f) o += w * op[(static_cast<long>(s) * a.d_c + c0 + c) * H];
-      }
-      tile[c][h] = o * inv_z;
+    // 32 independent loads per split keep enough requests in flight
+    float acc[kCombCols];
+#pragma unroll
+    for (int c = 0; c < kCombCols; ++c) acc[c] = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float w = cw[s * H + h];
+      const float* os = op + (static_cast<long>(s) * a.d_c + c0) * H;
+#pragma unroll
+      for (int c = 0; c < kCombCols; ++c)
+        if (c0 + c < a.d_c) acc[c] += w * os[static_cast<long>(c) * H];
     }
+#pragma unroll
+    for (int c = 0; c < kCombCols; ++c) tile[c][h] = acc[c] * inv_z;
   }
   __syncthreads();
   // o_lat[b][hh][c0 + cc]: a warp writes one head row of 32 columns per step

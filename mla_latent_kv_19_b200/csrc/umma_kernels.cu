@@ -2,6 +2,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <map>
 #include <mutex>
 
 #include "decode_umma.cuh"
@@ -40,21 +41,6 @@ cudaError_t make_map_rows_chunked(CUtensorMap* map, const void* base, uint64_t r
   const cuuint32_t box[3] = {64, box_rows, box_chunks};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
-// 2-D bf16 tensor map, 128-byte swizzle, box = box_cols x box_rows.
-cudaError_t make_map_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
-                          uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (fn == nullptr) return cudaErrorNotSupported;
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_cols, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
@@ -105,23 +91,41 @@ cudaError_t launch_decode_umma(const mla_ctx* h, const DecodeArgs& a, cudaStream
 
 namespace {
 
-constexpr int kOProjSplits = 7;      // K split of W_O: 40 row tiles x 7 = 280 CTAs, two per SM
-constexpr int kGemmStages = 5;
+constexpr int kOProjSplits = 3;      // K split of W_O: 40 row tiles x 3 = 120 CTAs, one per SM
 
 int padded_n(int batch) { return (batch + 15) / 16 * 16; }
 
-size_t gemm_smem_bytes(int n, int stages) {
-  return static_cast<size_t>(stages) * (gemm::kM * gemm::kKc * 2 + n * gemm::kKc * 2) +
-         8 * (2 * stages + 2) + 16 + 1024;
+size_t gemm_smem_bytes(const gemm::Params& p) {
+  return static_cast<size_t>(p.stages) *
+             (gemm::kM * gemm::kKc * 2 * p.kcs + p.n * gemm::kKc * 2 * p.kcs) +
+         8 * (2 * p.stages + 2) + 16 + 1024;
+}
+
+// Raise a kernel's dynamic shared-memory limit once (per process) to the
+// largest size requested so far; launches then pay no driver call.
+// (keyed by the kernel's address: every instantiation of a kernel template has
+// the same function type).
+template <typename K>
+cudaError_t ensure_smem_limit(K kernel, size_t bytes) {
+  static std::mutex mu;
+  static std::map<const void*, size_t> current;
+  std::lock_guard<std::mutex> lock(mu);
+  size_t& cur = current[reinterpret_cast<const void*>(kernel)];
+  if (bytes <= cur) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(bytes));
+  if (e == cudaSuccess) cur = bytes;
+  return e;
 }
 
 template <bool kAMn, gemm::Epi kEpi>
-cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tx, const gemm::Params& p,
-                        dim3 grid, cudaStream_t s) {
-  const size_t smem = gemm_smem_bytes(p.n, p.stages);
-  cudaError_t e = cudaFuncSetAttribute(gemm::gemm_wt_kernel<kAMn, kEpi>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tx, gemm::Params p, dim3 grid,
+                        cudaStream_t s) {
+  // as many stages as requested that fit in shared memory (larger batches: fewer)
+  while (p.stages > 2 && gemm_smem_bytes(p) > 232448) --p.stages;
+  const size_t smem = gemm_smem_bytes(p);
+  if (smem > 232448) return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem_limit(gemm::gemm_wt_kernel<kAMn, kEpi>, smem);
   if (e != cudaSuccess) return e;
   gemm::gemm_wt_kernel<kAMn, kEpi><<<grid, 256, smem, s>>>(ta, tx, p);
   note_launches(1);
@@ -144,12 +148,14 @@ bool umma_absorb_supported(const mla_ctx* h, int batch) {
 cudaError_t launch_absorb_umma(const mla_ctx* h, const AbsorbArgs& a, cudaStream_t s) {
   const int H = a.num_heads, n = padded_n(a.batch);
   CUtensorMap ta, tx;
-  // W_UK viewed as [H*d_nope rows (k)][d_c cols (c)], read MN-major in 64x64 boxes
-  cudaError_t e = make_map_bf16(&ta, a.w_uk, a.d_c, static_cast<uint64_t>(H) * a.d_nope, a.d_c * 2, 64, 64);
+  // W_UK [H*d_nope rows (k)][d_c columns (c)], read MN-major: a box is 128 rows of K
+  // by two 64-column slices of one 128-wide M tile
+  cudaError_t e = make_map_rows_chunked(&ta, a.w_uk, static_cast<uint64_t>(H) * a.d_nope, a.d_c * 2,
+                                        a.d_c / gemm::kKc, 2 * gemm::kKc, 2);
   if (e != cudaSuccess) return e;
-  // q_nope viewed as [B rows][H*d_nope cols]
-  e = make_map_bf16(&tx, a.q_nope, static_cast<uint64_t>(H) * a.d_nope, a.batch,
-                    static_cast<uint64_t>(H) * a.d_nope * 2, 64, n);
+  // q_nope as [B rows][H*d_nope columns]
+  e = make_map_rows_chunked(&tx, a.q_nope, a.batch, static_cast<uint64_t>(H) * a.d_nope * 2,
+                            H * a.d_nope / gemm::kKc, n, 2);
   if (e != cudaSuccess) return e;
   gemm::Params p{};
   p.n = n;
@@ -157,9 +163,11 @@ cudaError_t launch_absorb_umma(const mla_ctx* h, const AbsorbArgs& a, cudaStream
   p.k_chunks = a.d_nope / gemm::kKc;
   p.k_split = 1;
   p.m_per_group = a.d_c;
+  p.mt_per_cta = a.d_c / gemm::kM;      // one CTA per head
+  p.kcs = 2;
   p.a_row_group = a.d_nope;
   p.x_col_group = a.d_nope;
-  p.stages = 2;
+  p.stages = 4;
   p.out = a.q_lat;
   p.out_ld = static_cast<long>(H) * (a.d_c + a.d_r);
   p.out_group = a.d_c + a.d_r;
@@ -172,7 +180,7 @@ cudaError_t launch_absorb_umma(const mla_ctx* h, const AbsorbArgs& a, cudaStream
   p.max_position = a.max_position;
   p.err = a.err;
   p.wait_limit = h->wait_limit;
-  return launch_gemm<true, gemm::Epi::kAbsorb>(ta, tx, p, dim3(H * (a.d_c / gemm::kM), 1), s);
+  return launch_gemm<true, gemm::Epi::kAbsorb>(ta, tx, p, dim3(H, 1), s);
 }
 
 bool umma_out_proj_supported(const mla_ctx* h, int batch) {
@@ -191,10 +199,11 @@ cudaError_t launch_out_proj_umma(const mla_ctx* h, const OutProjArgs& a, void* e
   // o[b][h][v] = W_UV[h] o_lat[b][h]
   {
     CUtensorMap ta, tx;
-    cudaError_t e = make_map_bf16(&ta, a.w_uv, a.d_c, static_cast<uint64_t>(H) * a.d_v, a.d_c * 2, 64, 128);
+    cudaError_t e = make_map_rows_chunked(&ta, a.w_uv, static_cast<uint64_t>(H) * a.d_v, a.d_c * 2,
+                                          a.d_c / gemm::kKc, gemm::kM, 2);
     if (e != cudaSuccess) return e;
-    e = make_map_bf16(&tx, a.o_lat, static_cast<uint64_t>(H) * a.d_c, a.batch,
-                      static_cast<uint64_t>(H) * a.d_c * 2, 64, n);
+    e = make_map_rows_chunked(&tx, a.o_lat, a.batch, static_cast<uint64_t>(H) * a.d_c * 2,
+                              H * a.d_c / gemm::kKc, n, 2);
     if (e != cudaSuccess) return e;
     gemm::Params p{};
     p.n = n;
@@ -202,6 +211,8 @@ cudaError_t launch_out_proj_umma(const mla_ctx* h, const OutProjArgs& a, void* e
     p.k_chunks = a.d_c / gemm::kKc;
     p.k_split = 1;
     p.m_per_group = a.d_v;
+    p.mt_per_cta = 1;
+    p.kcs = 2;
     p.a_row_group = a.d_v;
     p.x_col_group = a.d_c;
     p.stages = 4;
@@ -217,9 +228,9 @@ cudaError_t launch_out_proj_umma(const mla_ctx* h, const OutProjArgs& a, void* e
   float* part = static_cast<float*>(extra);
   {
     CUtensorMap ta, tx;
-    cudaError_t e = make_map_bf16(&ta, a.w_o, kdim, a.d_model, kdim * 2, 64, 128);
+    cudaError_t e = make_map_rows_chunked(&ta, a.w_o, a.d_model, kdim * 2, kdim / gemm::kKc, gemm::kM, 2);
     if (e != cudaSuccess) return e;
-    e = make_map_bf16(&tx, a.o, kdim, a.batch, kdim * 2, 64, n);
+    e = make_map_rows_chunked(&tx, a.o, a.batch, kdim * 2, kdim / gemm::kKc, n, 2);
     if (e != cudaSuccess) return e;
     gemm::Params p{};
     p.n = n;
@@ -227,9 +238,11 @@ cudaError_t launch_out_proj_umma(const mla_ctx* h, const OutProjArgs& a, void* e
     p.k_chunks = static_cast<int>(kdim / gemm::kKc);
     p.k_split = kOProjSplits;
     p.m_per_group = a.d_model;
+    p.mt_per_cta = 1;
+    p.kcs = 2;
     p.a_row_group = 0;
     p.x_col_group = 0;
-    p.stages = kGemmStages;
+    p.stages = 5;
     p.out = part;
     p.out_ld = a.d_model;
     p.out_group = 0;

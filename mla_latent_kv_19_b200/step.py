@@ -160,6 +160,26 @@ class DecodeStep:
         self.decode_combine(stream)
         self.out_proj(stream)
 
+    # -- CUDA graphs of the step (the C-ABI calls neither allocate nor sync) --
+    def capture(self) -> None:
+        """Record one CUDA graph per stage and one for the whole step.  Call after
+        an ordinary run() (first calls configure kernels).  Replays reuse the
+        buffers of this object: refresh inputs in place (copy_) between replays."""
+        torch.cuda.synchronize(self.device)
+        self.stage_graphs = []
+        for fn in (self.append, self.absorb, self.decode_partial, self.decode_combine, self.out_proj):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            self.stage_graphs.append(g)
+        self.step_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.step_graph):
+            self.run()
+        torch.cuda.synchronize(self.device)
+
+    def replay(self) -> None:
+        self.step_graph.replay()
+
     def outputs(self) -> Dict[str, np.ndarray]:
         torch.cuda.synchronize(self.device)
         f = lambda t: t.float().cpu().numpy().astype(np.float64)

@@ -99,3 +99,16 @@ def test_create_without_device_reports_cuda_error():
         pytest.skip("a GPU is present")
     st, h = _create(_cfg())
     assert st == -8 and not h.value
+
+
+def test_binding_counts_pages_from_the_cache_size():
+    """The page count handed to the library (its bounds check on page-table
+    entries) comes from the cache's size, whatever the tensor's shape."""
+    import types
+
+    import torch
+    h = types.SimpleNamespace(cfg=types.SimpleNamespace(block_size=64, d_c=512, d_r=64))
+    assert m._num_blocks(h, torch.empty(10 * 64, 576, dtype=torch.bfloat16)) == 10
+    assert m._num_blocks(h, torch.empty(7, 64, 576, dtype=torch.uint8)) == 7
+    with pytest.raises(ValueError):
+        m._num_blocks(h, torch.empty(100, 576))
