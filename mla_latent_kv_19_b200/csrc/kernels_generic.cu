@@ -403,11 +403,12 @@ cudaError_t launch_decode_generic(const DecodeArgs& a, int act_dtype, int cache_
 // split merge by log-sum-exp
 // ---------------------------------------------------------------------------
 
-// One CTA per (sequence b, chunk of 32 latent columns); thread = head.  Reads
+// One CTA per (sequence b, chunk of 16 latent columns); thread = head.  Reads
 // o_part[b][s][c][h] (coalesced over heads), merges the splits with weights
 // exp(lse_s - lse), transposes through shared memory and writes o_lat[b][h][c]
-// rows of 32 contiguous columns.
-constexpr int kCombCols = 32;
+// rows of 16 contiguous columns.  16 columns per thread keep the register count
+// low enough for several CTAs per SM and many loads in flight.
+constexpr int kCombCols = 16;
 
 template <typename T>
 __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
@@ -416,40 +417,41 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
   const int b = blockIdx.x, c0 = blockIdx.y * kCombCols;
   const int S = a.num_splits, H = a.num_heads;
   const int h = threadIdx.x;                  // blockDim.x == 128 >= H
-  float inv_z = 0.f;
   if (h < H) {
     const float* lp = a.lse_part + static_cast<long>(b) * S * H + h;
     float m = -INFINITY;
+#pragma unroll 4
     for (int s = 0; s < S; ++s) m = fmaxf(m, lp[static_cast<long>(s) * H]);
     float z = 0.f;
+#pragma unroll 4
     for (int s = 0; s < S; ++s) {
       const float w = (m == -INFINITY) ? 0.f : __expf(lp[static_cast<long>(s) * H] - m);
       cw[s * H + h] = w;
       z += w;
     }
-    inv_z = z > 0.f ? 1.f / z : 0.f;
+    const float inv_z = z > 0.f ? 1.f / z : 0.f;
     if (blockIdx.y == 0 && a.lse != nullptr)
       a.lse[static_cast<long>(b) * H + h] = z > 0.f ? m + __logf(z) : -INFINITY;
-    const float* op = a.o_part + static_cast<long>(b) * S * a.d_c * H + h;
-    // 32 independent loads per split keep enough requests in flight
+    const float* op = a.o_part + (static_cast<long>(b) * S * a.d_c + c0) * H + h;
     float acc[kCombCols];
 #pragma unroll
     for (int c = 0; c < kCombCols; ++c) acc[c] = 0.f;
+    const int nc = min(kCombCols, a.d_c - c0);
     for (int s = 0; s < S; ++s) {
       const float w = cw[s * H + h];
-      const float* os = op + (static_cast<long>(s) * a.d_c + c0) * H;
+      const float* os = op + static_cast<long>(s) * a.d_c * H;
 #pragma unroll
       for (int c = 0; c < kCombCols; ++c)
-        if (c0 + c < a.d_c) acc[c] += w * os[static_cast<long>(c) * H];
+        if (c < nc) acc[c] += w * os[c * H];
     }
 #pragma unroll
     for (int c = 0; c < kCombCols; ++c) tile[c][h] = acc[c] * inv_z;
   }
   __syncthreads();
-  // o_lat[b][hh][c0 + cc]: a warp writes one head row of 32 columns per step
+  // o_lat[b][hh][c0 + cc]: each half warp writes one head row of 16 columns
   T* out = reinterpret_cast<T*>(a.o_lat) + static_cast<long>(b) * H * a.d_c;
-  const int cc = threadIdx.x & 31;
-  for (int hh = threadIdx.x >> 5; hh < H; hh += 4)
+  const int cc = threadIdx.x & 15;
+  for (int hh = threadIdx.x >> 4; hh < H; hh += 8)
     if (c0 + cc < a.d_c) out[static_cast<long>(hh) * a.d_c + c0 + cc] = cvt_out<T>(tile[cc][hh]);
 }
 
