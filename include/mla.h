@@ -29,7 +29,9 @@
  *   q_lat, o_lat, y, weights) use the handle's act_dtype; the cache uses
  *   cache_dtype.
  * - Device pointers to activations, weights, caches and workspaces must be
- *   16-byte aligned (vector and TMA access); int32 and fp32-scale arrays 4-byte.
+ *   16-byte aligned (vector and TMA access); int32 arrays 4-byte; the fp32
+ *   cache_scale array 4-byte for the append calls and 16-byte for the decode
+ *   calls (a page's 64 scales are fetched by one bulk copy).
  * - Return value: MLA_OK (0) or a negative mla_status_t.  A call that returns
  *   an error has launched nothing.  Invalid page-table entries or positions
  *   found by a kernel are reported through the device error word, read by
@@ -188,9 +190,10 @@ MLA_API int mla_decode(mla_handle_t h, const void* q_lat, const void* cache, con
 /* The two halves of mla_decode, for callers that time or schedule them
  * separately.  mla_decode_partial writes the workspace; mla_decode_combine
  * reads it (same batch / num_splits / max_seq_len) and writes o_lat and lse.
- * Workspace layout (fp32): o_part [batch][S][d_c][H] (heads innermost) followed,
- * at the next 256-byte boundary, by lse_part [batch][S][H]; an empty range
- * stores lse_part = -inf, o_part = 0. */
+ * Workspace layout (fp32): o_part [batch][S][d_c/4][H][4] (groups of four
+ * latent columns, heads next: o_part[b][s][c/4][h][c%4]) followed, at the next
+ * 256-byte boundary, by lse_part [batch][S][H]; an empty range stores
+ * lse_part = -inf, o_part = 0. */
 MLA_API int mla_decode_partial(mla_handle_t h, const void* q_lat, const void* cache,
                        const float* cache_scale, int32_t num_blocks, const int32_t* block_table,
                        int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t batch,

@@ -113,6 +113,18 @@ def _num_blocks(h: "Handle", cache) -> int:
     return n
 
 
+def _scale_ptr(h: "Handle", cache, cache_scale) -> Optional[int]:
+    """Pointer of an fp8 cache's per-token scales, after checking that it holds
+    one fp32 per cache row (the kernels read a page's scales by page index)."""
+    if cache_scale is None:
+        return None
+    rows = _num_blocks(h, cache) * h.cfg.block_size
+    if cache_scale.dtype != torch.float32 or cache_scale.numel() < rows:
+        raise ValueError(f"cache_scale must hold {rows} fp32 values (one per cache row), "
+                         f"got {cache_scale.numel()} of {cache_scale.dtype}")
+    return _ptr(cache_scale)
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -164,7 +176,7 @@ def mla_cache_append(h: Handle, c_kv, k_r, pos, block_table, cache, cache_scale=
     batch = block_table.shape[0] if batch is None else batch
     _check("mla_cache_append", lib.mla_cache_append(
         h.ptr, _ptr(c_kv), _ptr(k_r), _ptr(seq_idx), _ptr(pos), n, _ptr(block_table),
-        block_table.shape[1], batch, _ptr(cache), _ptr(cache_scale), _num_blocks(h, cache), _stream(stream)))
+        block_table.shape[1], batch, _ptr(cache), _scale_ptr(h, cache, cache_scale), _num_blocks(h, cache), _stream(stream)))
 
 
 def mla_kv_project_append(h: Handle, x, w_dkv, w_kr, pos, block_table, cache, cache_scale=None,
@@ -173,7 +185,7 @@ def mla_kv_project_append(h: Handle, x, w_dkv, w_kr, pos, block_table, cache, ca
     batch = block_table.shape[0] if batch is None else batch
     _check("mla_kv_project_append", lib.mla_kv_project_append(
         h.ptr, _ptr(x), _ptr(w_dkv), _ptr(w_kr), _ptr(seq_idx), _ptr(pos), n, _ptr(block_table),
-        block_table.shape[1], batch, _ptr(cache), _ptr(cache_scale), _num_blocks(h, cache), _stream(stream)))
+        block_table.shape[1], batch, _ptr(cache), _scale_ptr(h, cache, cache_scale), _num_blocks(h, cache), _stream(stream)))
 
 
 def mla_absorb_q(h: Handle, q_nope, q_pe, pos, w_uk, q_lat, stream=None) -> None:
@@ -193,7 +205,7 @@ def mla_decode_workspace_bytes(h: Handle, batch: int, num_splits: int, max_seq_l
 def mla_decode(h: Handle, q_lat, cache, cache_scale, block_table, seq_lens, max_seq_len: int,
                num_splits: int, workspace, o_lat, lse=None, stream=None) -> None:
     _check("mla_decode", lib.mla_decode(
-        h.ptr, _ptr(q_lat), _ptr(cache), _ptr(cache_scale), _num_blocks(h, cache), _ptr(block_table),
+        h.ptr, _ptr(q_lat), _ptr(cache), _scale_ptr(h, cache, cache_scale), _num_blocks(h, cache), _ptr(block_table),
         block_table.shape[1], _ptr(seq_lens), seq_lens.shape[0], max_seq_len, num_splits,
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(o_lat), _ptr(lse),
         _stream(stream)))
@@ -202,7 +214,7 @@ def mla_decode(h: Handle, q_lat, cache, cache_scale, block_table, seq_lens, max_
 def mla_decode_partial(h: Handle, q_lat, cache, cache_scale, block_table, seq_lens,
                        max_seq_len: int, num_splits: int, workspace, stream=None) -> None:
     _check("mla_decode_partial", lib.mla_decode_partial(
-        h.ptr, _ptr(q_lat), _ptr(cache), _ptr(cache_scale), _num_blocks(h, cache), _ptr(block_table),
+        h.ptr, _ptr(q_lat), _ptr(cache), _scale_ptr(h, cache, cache_scale), _num_blocks(h, cache), _ptr(block_table),
         block_table.shape[1], _ptr(seq_lens), seq_lens.shape[0], max_seq_len, num_splits,
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
@@ -220,7 +232,7 @@ def mla_decode_noalloc(h: Handle, q_lat, cache, cache_scale, block_table, seq_le
     fixed 32 MiB device array inside the library (for callers that cannot
     allocate device memory).  Overlapping calls on one device race on it."""
     _check("mla_decode_noalloc", lib.mla_decode_noalloc(
-        h.ptr, _ptr(q_lat), _ptr(cache), _ptr(cache_scale), _num_blocks(h, cache), _ptr(block_table),
+        h.ptr, _ptr(q_lat), _ptr(cache), _scale_ptr(h, cache, cache_scale), _num_blocks(h, cache), _ptr(block_table),
         block_table.shape[1], _ptr(seq_lens), seq_lens.shape[0], max_seq_len, num_splits,
         _ptr(o_lat), _ptr(lse), _stream(stream)))
 

@@ -291,7 +291,7 @@ int mla_decode_partial(mla_handle_t h, const void* q_lat, const void* cache,
   if (static_cast<long>(max_seq_len) > static_cast<long>(max_blocks_per_seq) * h->cfg.block_size)
     return MLA_ERR_INVALID_ARG;
   if (!aligned(q_lat, 16) || !aligned(cache, 16) || !aligned(block_table, 4) ||
-      !aligned(seq_lens, 4) || (cache_scale && !aligned(cache_scale, 4)))
+      !aligned(seq_lens, 4) || (cache_scale && !aligned(cache_scale, 16)))
     return MLA_ERR_ALIGNMENT;
   DecodeArgs a{};
   a.q_lat = q_lat;

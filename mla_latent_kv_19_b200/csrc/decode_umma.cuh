@@ -24,8 +24,9 @@
 //     TMEM lane quadrant each, one head per thread) run the online softmax and
 //     write P (bf16, UMMA K-major swizzled layout) plus the rescale factors
 //     into the page's own slot -- its K data is no longer needed -- and one
-//     thread ships that message to CTA 1 with a single bulk copy; CTA 1 frees
-//     the slot once its P V has consumed the message.
+//     thread ships that message to CTA 1 with a single bulk copy (into one of
+//     three P buffers, once P V has finished reading that buffer's previous
+//     message); CTA 1 frees the slot as soon as the message has landed.
 //   CTA 1 ("value"):  O accumulates in TMEM columns 0..511; the same pages'
 //     first 512 columns stream through a 2-stage ring, one 64 KB TMA request
 //     per page (an L2 hit after CTA 0's read); P V is issued as two N = 256
@@ -65,6 +66,15 @@ constexpr int kPBytes = kH * kTok * 2;                 // 16384
 constexpr int kPMsgBytes = kPBytes + kH * 4 + 16;      // P + alpha[128] + flag[4] = 16912
 constexpr int kPBufStride = 17 * 1024;                 // keeps every P tile 1024-byte aligned
 constexpr int kMaxTablePages = 512;                    // pages of a split kept in shared memory
+constexpr int kPrefetchPages = 4;                      // L2 prefetch distance ahead of the ring's loads
+// e4m3 cache: a page is 64 rows x 576 code bytes, contiguous in the pool, plus
+// 64 fp32 per-token scales
+constexpr int kPageF8Bytes = kTok * kD;                // 36864
+constexpr int kF8InSlot = kSlotBytes - kPageF8Bytes;   // codes land in a slot's upper half
+constexpr int kF8InStage = kVStageBytes - kPageF8Bytes;
+constexpr int kScaleBytes = kTok * 4;
+constexpr int kF8UnitsK = kPageF8Bytes / 8 / 128;      // 36 eight-code units per converter thread
+constexpr int kF8UnitsV = kTok * kDc / 8 / 128;        // 32 (V: first 512 columns)
 
 // CTA 0 map
 constexpr int kOffRing = 0;
@@ -85,9 +95,13 @@ enum Bar {
   kVFull = kStg + 2, kVEmpty = kVFull + kVStages,                       // CTA 1
   kPFull = kVEmpty + kVStages, kPVDone = kPFull + kPBufs,
   kCorrReq = kPVDone + 2, kCorrDone = kCorrReq + 1, kOFull = kCorrDone + 1, kFin = kOFull + 1,
-  kDrain = kFin + 1, kNumBars = kDrain + 1
+  kDrain = kFin + 1,
+  kCvtLd = kDrain + 1, kCvtDone = kCvtLd + 1, kVCvt = kCvtDone + kSlots,  // e4m3 converters
+  kPBufFree = kVCvt + kVStages,                                          // CTA 0: CTA 1's P buffers
+  kNumBars = kPBufFree + kPBufs
 };
-constexpr int kOffBar = kRegionEnd;
+constexpr int kOffScale = kRegionEnd;                  // CTA 0: per-token scales [3 slots][64]
+constexpr int kOffBar = kOffScale + kSlots * kScaleBytes;
 // misc words: [0] tmem base, [1] abort, [2] corr tile, [3] P messages CTA 0 sent
 // (written by CTA 0 into CTA 1), [4] messages CTA 1 consumed, [5] messages it armed
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -143,7 +157,26 @@ __device__ __forceinline__ int valid_tokens(const Split& s, int page, int t) {
   return page < 0 ? 0 : min(kTok, s.len - (s.p0 + t) * kTok);
 }
 
-__global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
+// Two e4m3 codes (low byte first) to two bf16 values.  Exact: an e4m3 value has
+// at most 4 significant bits and its exponent range lies inside bf16's.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
+  const float2 f = __half22float2(__half2(h));
+  const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 v) {
+  return make_uint4(e4m3x2_to_bf16x2(v.x), e4m3x2_to_bf16x2(v.x >> 16), e4m3x2_to_bf16x2(v.y),
+                    e4m3x2_to_bf16x2(v.y >> 16));
+}
+
+// Threads per CTA: 8 warps, plus 4 converter warps with an e4m3 cache.
+template <bool kFp8>
+constexpr int threads() { return kFp8 ? 384 : 256; }
+
+template <bool kFp8>
+__global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
     decode_umma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                        const __grid_constant__ CUtensorMap qmap, const DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -207,6 +240,10 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
     ptx::mbar_init(bar(kOFull), 1);
     ptx::mbar_init(bar(kFin), 128);
     ptx::mbar_init(bar(kDrain), 1);
+    ptx::mbar_init(bar(kCvtLd), 128);
+    for (int i = 0; i < kSlots; ++i) ptx::mbar_init(bar(kCvtDone + i), 128);
+    for (int i = 0; i < kVStages; ++i) ptx::mbar_init(bar(kVCvt + i), 128);
+    for (int i = 0; i < kPBufs; ++i) ptx::mbar_init(bar(kPBufFree + i), 1);
     misc[1] = 0u;
     misc[2] = 0u;
     misc[3] = 0u;
@@ -231,20 +268,44 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
       if (lane == 0) {
         // TMA producer over the ring: 2 halves of Q, then one request per page.  A
         // page's slot comes back when CTA 1 has consumed the P message in it.
-        ptx::prefetch_tmap(&kmap);
+        if (!kFp8) ptx::prefetch_tmap(&kmap);
         ptx::prefetch_tmap(&qmap);
+        // pages are fetched into L2 a few tiles before their slot frees, so that
+        // the slot's own load is an L2 hit
+        auto prefetch_page = [&](int t) {
+          if (t >= sp.ntiles) return;
+          const long pg = max(page_at(a, sp, table, t), 0);
+          if (kFp8) {
+            ptx::prefetch_l2(static_cast<const uint8_t*>(a.cache) + pg * kPageF8Bytes, kPageF8Bytes);
+            ptx::prefetch_l2(a.cache_scale + pg * kTok, kScaleBytes);
+          } else {
+            ptx::prefetch_l2(static_cast<const uint8_t*>(a.cache) + pg * kSlotBytes, kSlotBytes);
+          }
+        };
+        for (int t = 0; t < kPrefetchPages; ++t) prefetch_page(t);
         const int total = kQLoads + sp.ntiles;
         int issued = 0;
         for (int n = 0; n < total; ++n) {
           const int slot = n % kSlots;
           if (!wait_remote(bar(kEmpty + slot), ((n / kSlots) & 1) ^ 1)) break;
-          ptx::mbar_arrive_expect_tx(bar(kFull + slot), kSlotBytes);
           const uint32_t dst = sb + kOffRing + slot * kSlotBytes;
           if (n < kQLoads) {
+            ptx::mbar_arrive_expect_tx(bar(kFull + slot), kSlotBytes);
             ptx::tma_load_3d(dst, &qmap, bar(kFull + slot), 0, sp.b * kH + 64 * n, 0);
           } else {
-            const int pg = page_at(a, sp, table, n - kQLoads);
-            ptx::tma_load_3d(dst, &kmap, bar(kFull + slot), 0, (pg < 0 ? 0 : pg) * kTok, 0);
+            const int pg = max(page_at(a, sp, table, n - kQLoads), 0);
+            prefetch_page(n - kQLoads + kPrefetchPages);
+            if (kFp8) {
+              // the page's codes (contiguous) into the slot's upper half, its scales aside
+              ptx::mbar_arrive_expect_tx(bar(kFull + slot), kPageF8Bytes + kScaleBytes);
+              ptx::bulk_load(dst + kF8InSlot, static_cast<const uint8_t*>(a.cache) + static_cast<long>(pg) * kPageF8Bytes,
+                             kPageF8Bytes, bar(kFull + slot));
+              ptx::bulk_load(sb + kOffScale + slot * kScaleBytes, a.cache_scale + static_cast<long>(pg) * kTok,
+                             kScaleBytes, bar(kFull + slot));
+            } else {
+              ptx::mbar_arrive_expect_tx(bar(kFull + slot), kSlotBytes);
+              ptx::tma_load_3d(dst, &kmap, bar(kFull + slot), 0, pg * kTok, 0);
+            }
           }
           issued = n + 1;
         }
@@ -264,7 +325,10 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
             const int n = kQLoads + t;
             const int slot = n % kSlots;
             if (!wait_local(bar(kSEmpty + i), ((t >> 1) & 1) ^ 1)) break;
-            if (!wait_local(bar(kFull + slot), (n / kSlots) & 1)) break;
+            // the page in bf16: as landed, or once the converters have expanded its codes
+            if (!(kFp8 ? wait_local(bar(kCvtDone + slot), (t / kSlots) & 1)
+                       : wait_local(bar(kFull + slot), (n / kSlots) & 1)))
+              break;
             ptx::tc_fence_after();
             // S[i] = Q K^T over the 9 chunks of K = 576, one page (N = 64) per MMA
             const uint32_t d = tmem + kColS + 64u * i;
@@ -284,7 +348,7 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
         drain(bar(kDrain), 0);
       }
       __syncwarp();
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < 8) {
       // softmax warpgroup: thread = head row r, TMEM lane quadrant q
       const int q = warp & 3;
       const int r = q * 32 + lane;
@@ -335,12 +399,21 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
         ptx::tc_fence_before();
         ptx::mbar_arrive(bar(kSEmpty + i));
         const int valid = valid_tokens(sp, page_at(a, sp, table, t), t);
+        const int slot = (kQLoads + t) % kSlots;
+        // e4m3 cache: row j is scale_j times its codes, so score j is scale_j times
+        // the score against the codes (the scales came in with the page)
+        const float* scl = reinterpret_cast<const float*>(smem + kOffScale + slot * kScaleBytes);
+        if (kFp8) {
+          w = wait_local(bar(kFull + slot), ((kQLoads + t) / kSlots) & 1);
+          if (!__all_sync(0xffffffffu, w)) break;
+        }
         float x[64];
         float m_tile = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          x[j] = j < valid ? __uint_as_float(s0[j]) * sl2 : -INFINITY;
-          x[j + 32] = j + 32 < valid ? __uint_as_float(s1[j]) * sl2 : -INFINITY;
+          const float f0 = kFp8 ? sl2 * scl[j] : sl2, f1 = kFp8 ? sl2 * scl[j + 32] : sl2;
+          x[j] = j < valid ? __uint_as_float(s0[j]) * f0 : -INFINITY;
+          x[j + 32] = j + 32 < valid ? __uint_as_float(s1[j]) * f1 : -INFINITY;
           m_tile = fmaxf(m_tile, fmaxf(x[j], x[j + 32]));
         }
         const bool resc = m_tile > m_used + kRescaleThreshold;
@@ -356,13 +429,20 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
         for (int j = 0; j < 32; ++j) {
           const float p0 = live ? ptx::ex2(x[2 * j] - m_used) : 0.f;
           const float p1 = live ? ptx::ex2(x[2 * j + 1] - m_used) : 0.f;
-          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-          psum += __low2float(pb) + __high2float(pb);
+          __nv_bfloat162 pb;
+          if (kFp8) {
+            // the P V operand carries scale_j (V holds the codes); l sums the weights
+            psum += p0 + p1;
+            pb = __floats2bfloat162_rn(2 * j < valid ? p0 * scl[2 * j] : 0.f,
+                                       2 * j + 1 < valid ? p1 * scl[2 * j + 1] : 0.f);
+          } else {
+            pb = __floats2bfloat162_rn(p0, p1);
+            psum += __low2float(pb) + __high2float(pb);
+          }
           pk[j] = *reinterpret_cast<const uint32_t*>(&pb);
         }
         l = l * alpha + psum;
         // the message goes into this page's ring slot: S(t) has consumed its K data
-        const int slot = (kQLoads + t) % kSlots;
         uint8_t* msg = smem + kOffRing + slot * kSlotBytes;
         uint8_t* prow = msg + r * 128;
 #pragma unroll
@@ -375,8 +455,10 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
         ptx::fence_proxy_async_cta();              // generic writes -> bulk-copy reads
         ptx::mbar_arrive(bar(kStg + i));
         if (r == 0) {
-          // every row of the message is written: ship it to CTA 1 in one bulk copy
-          if (wait_local(bar(kStg + i), (t >> 1) & 1)) {
+          // every row of the message is written and CTA 1's buffer t % 3 is no longer
+          // read by P V(t - 3): ship the message in one bulk copy
+          if (wait_local(bar(kStg + i), (t >> 1) & 1) &&
+              wait_remote(bar(kPBufFree + t % kPBufs), ((t / kPBufs) & 1) ^ 1)) {
             ptx::bulk_copy_to_peer(rP + (t % kPBufs) * kPBufStride, sb + kOffRing + slot * kSlotBytes,
                                    kPMsgBytes, rPFull + 8u * (t % kPBufs));
             ++sent;
@@ -389,21 +471,55 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
       ptx::st_cluster_u32(rL + r * 4, __float_as_uint(l));
       ptx::mbar_arrive_remote(rFin);
       if (r == 0) ptx::st_cluster_u32(ptx::mapa(sb + kOffMisc + 12, 1), sent);
+    } else if (kFp8 && warp >= 8) {
+      // converters: expand a landed page's e4m3 codes, in place, into the bf16
+      // chunk-major swizzled layout S = Q K^T reads.  Every thread holds its
+      // share of the codes in registers before any thread writes (the bf16 page
+      // covers the codes' bytes).
+      const int ct = static_cast<int>(threadIdx.x) - 256;
+#pragma unroll 1
+      for (int t = 0; t < sp.ntiles; ++t) {
+        const int n = kQLoads + t, slot = n % kSlots;
+        bool ok = wait_local(bar(kFull + slot), (n / kSlots) & 1);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        uint8_t* page = smem + kOffRing + slot * kSlotBytes;
+        uint2 u[kF8UnitsK];
+#pragma unroll
+        for (int k = 0; k < kF8UnitsK; ++k)
+          u[k] = *reinterpret_cast<const uint2*>(page + kF8InSlot + (k * 128 + ct) * 8);
+        ptx::mbar_arrive(bar(kCvtLd));
+        ok = wait_local(bar(kCvtLd), t & 1);
+        if (!__all_sync(0xffffffffu, ok)) break;
+#pragma unroll
+        for (int k = 0; k < kF8UnitsK; ++k) {
+          const int g = k * 128 + ct, row = g / 72, cu = g - row * 72;
+          *reinterpret_cast<uint4*>(page + (cu >> 3) * kChunkInSlot + row * 128 + (((cu & 7) ^ (row & 7)) << 4)) =
+              e4m3x8_to_bf16x8(u[k]);
+        }
+        ptx::fence_proxy_async_cta();              // generic writes -> tensor-core reads
+        ptx::mbar_arrive(bar(kCvtDone + slot));
+      }
     }
   } else {
     // =========================== CTA 1: values ===========================
     if (warp == 0) {
       if (lane == 0) {
         // TMA producer: first 512 columns of the same pages
-        ptx::prefetch_tmap(&vmap);
+        if (!kFp8) ptx::prefetch_tmap(&vmap);
         int issued = 0;
         for (int t = 0; t < sp.ntiles; ++t) {
           const int st = t % kVStages;
           if (!wait_local(bar(kVEmpty + st), ((t / kVStages) & 1) ^ 1)) break;
-          const int pg = page_at(a, sp, table, t);
-          ptx::mbar_arrive_expect_tx(bar(kVFull + st), kVStageBytes);
-          ptx::tma_load_3d(sb + kOffV + st * kVStageBytes, &vmap, bar(kVFull + st), 0,
-                           (pg < 0 ? 0 : pg) * kTok, 0);
+          const int pg = max(page_at(a, sp, table, t), 0);
+          if (kFp8) {
+            ptx::mbar_arrive_expect_tx(bar(kVFull + st), kPageF8Bytes);
+            ptx::bulk_load(sb + kOffV + st * kVStageBytes + kF8InStage,
+                           static_cast<const uint8_t*>(a.cache) + static_cast<long>(pg) * kPageF8Bytes,
+                           kPageF8Bytes, bar(kVFull + st));
+          } else {
+            ptx::mbar_arrive_expect_tx(bar(kVFull + st), kVStageBytes);
+            ptx::tma_load_3d(sb + kOffV + st * kVStageBytes, &vmap, bar(kVFull + st), 0, pg * kTok, 0);
+          }
           issued = t + 1;
         }
         for (int t = max(0, issued - kVStages); t < issued; ++t)
@@ -417,16 +533,11 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
 #pragma unroll 1
       for (int t = 0; t < sp.ntiles; ++t) {
         const int st = t & 1, pbi = t % kPBufs;
-        if (lane == 0) {
-          ptx::mbar_arrive_expect_tx(bar(kPFull + pbi), kPMsgBytes);
-          misc[5] = static_cast<uint32_t>(t + 1);
-        }
-        bool ok = wait_local(bar(kVFull + st), (t >> 1) & 1);
+        bool ok = wait_local(bar((kFp8 ? kVCvt : kVFull) + st), (t >> 1) & 1);
         ok = ok && wait_remote(bar(kPFull + pbi), (t / kPBufs) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
-        if (lane == 0) misc[4] = static_cast<uint32_t>(t + 1);
         const int valid = valid_tokens(sp, page_at(a, sp, table, t), t);
-        if (valid < kTok) {
+        if (!kFp8 && valid < kTok) {
           // rows past the sequence end: zero them so that P = 0 meets finite V
           uint8_t* vs = smem + kOffV + st * kVStageBytes;
           const int n = (kTok - valid) * kVBoxes * 8;
@@ -476,19 +587,34 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
       }
       __syncwarp();
     } else if (warp == 2) {
-      // release: a finished P V frees its V stage here and, in CTA 0, the ring
-      // slot that carried its P message
+      // release: a finished P V frees its V stage and its P buffer (CTA 0 waits
+      // for the latter before shipping the next message into it)
       if (lane == 0) {
-        const uint32_t rEmpty = ptx::mapa(bar(kEmpty), 0);
+        const uint32_t rPBufFree = ptx::mapa(bar(kPBufFree), 0);
         for (int t = 0; t < sp.ntiles; ++t) {
           const int i = t & 1;
           if (!wait_local(bar(kPVDone + i), (t >> 1) & 1)) break;
           ptx::mbar_arrive(bar(kVEmpty + i));
+          ptx::mbar_arrive_remote(rPBufFree + 8u * (t % kPBufs));
+        }
+      }
+      __syncwarp();
+    } else if (warp == 3) {
+      // P receiver: arms each message's barrier, waits for the message to land and
+      // at once returns CTA 0's ring slot that carried it
+      if (lane == 0) {
+        const uint32_t rEmpty = ptx::mapa(bar(kEmpty), 0);
+        for (int t = 0; t < sp.ntiles; ++t) {
+          const int pbi = t % kPBufs;
+          ptx::mbar_arrive_expect_tx(bar(kPFull + pbi), kPMsgBytes);
+          misc[5] = static_cast<uint32_t>(t + 1);
+          if (!wait_remote(bar(kPFull + pbi), (t / kPBufs) & 1)) break;
+          misc[4] = static_cast<uint32_t>(t + 1);
           ptx::mbar_arrive_remote(rEmpty + 8u * ((kQLoads + t) % kSlots));
         }
       }
       __syncwarp();
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < 8) {
       // correction (rescale O rows on request) and epilogue
       const int q = warp & 3;
       const int r = q * 32 + lane;
@@ -524,14 +650,16 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
       bool ok = wait_local(bar(kOFull), 0);
       ok = ok && wait_remote(bar(kFin), 0);
       ok = __all_sync(0xffffffffu, ok);
-      // o_part[b][split][c][h]: for each column c the 32 lanes store 32 consecutive heads
-      float* obase = a.o_part + (static_cast<long>(sp.b) * a.num_splits + sp.split) * kDc * kH + r;
+      // o_part[b][split][c/4][h][c%4]: per group of four columns the 32 lanes store
+      // 32 consecutive heads' float4s (512 contiguous bytes)
+      float4* obase = reinterpret_cast<float4*>(a.o_part) +
+                      (static_cast<long>(sp.b) * a.num_splits + sp.split) * (kDc / 4) * kH + r;
       if (ok) {
         ptx::tc_fence_after();
         const float lsum = reinterpret_cast<const volatile float*>(smem + kOffLfin)[r];
         const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
         if (sp.ntiles == 0) {
-          for (int c = 0; c < kDc; ++c) obase[c * kH] = 0.f;
+          for (int g = 0; g < kDc / 4; ++g) obase[g * kH] = make_float4(0.f, 0.f, 0.f, 0.f);
         } else {
 #pragma unroll 1
           for (int c = 0; c < 16; ++c) {
@@ -539,10 +667,43 @@ __global__ void __launch_bounds__(256, 1) __cluster_dims__(2, 1, 1)
             ptx::tmem_ld32(tmem + lb + kColO + 32u * c, v);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) obase[(32 * c + e) * kH] = __uint_as_float(v[e]) * inv;
+            for (int e = 0; e < 8; ++e)
+              obase[(8 * c + e) * kH] = make_float4(__uint_as_float(v[4 * e]) * inv, __uint_as_float(v[4 * e + 1]) * inv,
+                                                    __uint_as_float(v[4 * e + 2]) * inv, __uint_as_float(v[4 * e + 3]) * inv);
           }
         }
         ptx::tc_fence_before();
+      }
+    } else if (kFp8 && warp >= 8) {
+      // converters: the first 512 columns of a landed page to bf16, in place, in
+      // the stage's chunk-major swizzled layout (the MN-major V operand); rows past
+      // the sequence end become zeros so that P = 0 meets finite V
+      const int ct = static_cast<int>(threadIdx.x) - 256;
+#pragma unroll 1
+      for (int t = 0; t < sp.ntiles; ++t) {
+        const int st = t % kVStages;
+        bool ok = wait_local(bar(kVFull + st), (t / kVStages) & 1);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const int valid = valid_tokens(sp, page_at(a, sp, table, t), t);
+        uint8_t* stage = smem + kOffV + st * kVStageBytes;
+        uint2 u[kF8UnitsV];
+#pragma unroll
+        for (int k = 0; k < kF8UnitsV; ++k) {
+          const int g = k * 128 + ct, row = g >> 6, cu = g & 63;
+          u[k] = row < valid ? *reinterpret_cast<const uint2*>(stage + kF8InStage + row * kD + cu * 8)
+                             : make_uint2(0u, 0u);
+        }
+        ptx::mbar_arrive(bar(kCvtLd));
+        ok = wait_local(bar(kCvtLd), t & 1);
+        if (!__all_sync(0xffffffffu, ok)) break;
+#pragma unroll
+        for (int k = 0; k < kF8UnitsV; ++k) {
+          const int g = k * 128 + ct, row = g >> 6, cu = g & 63;
+          *reinterpret_cast<uint4*>(stage + (cu >> 3) * kBoxBytes + row * 128 + (((cu & 7) ^ (row & 7)) << 4)) =
+              e4m3x8_to_bf16x8(u[k]);
+        }
+        ptx::fence_proxy_async_cta();
+        ptx::mbar_arrive(bar(kVCvt + st));
       }
     }
   }

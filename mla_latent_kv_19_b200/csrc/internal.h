@@ -63,7 +63,7 @@ struct DecodeArgs {
   const float* cache_scale;   // [num_blocks, block_size] (fp8)
   const int32_t* block_table; // [B, max_blocks]
   const int32_t* seq_lens;    // [B]
-  float* o_part;              // [B, S, H, d_c]
+  float* o_part;              // [B, S, d_c/4, H, 4]
   float* lse_part;            // [B, S, H]
   int* err;
   int32_t batch, num_heads, d_c, d_r, block_size, max_blocks, num_splits, num_blocks;

@@ -353,7 +353,8 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(DecodeArgs 
   }
   __syncthreads();
   const long part = (static_cast<long>(b) * a.num_splits + split) * a.num_heads;
-  const long obase = (static_cast<long>(b) * a.num_splits + split) * a.d_c;   // o_part[b][s][c][h]
+  // o_part[b][s][c/4][h][c%4]
+  float* obase = a.o_part + (static_cast<long>(b) * a.num_splits + split) * a.d_c * a.num_heads;
 #pragma unroll
   for (int jc = 0; jc < kGenColsPerThread; ++jc) {
     const int c = tid + jc * kGenThreads;
@@ -362,7 +363,7 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(DecodeArgs 
       for (int g = 0; g < kGenHeads; ++g) {
         if (g < nh) {
           const float l = ps[g];
-          a.o_part[(obase + c) * a.num_heads + h0 + g] = l > 0.f ? acc[g][jc] / l : 0.f;
+          obase[((c >> 2) * a.num_heads + h0 + g) * 4 + (c & 3)] = l > 0.f ? acc[g][jc] / l : 0.f;
         }
       }
     }
@@ -404,7 +405,7 @@ cudaError_t launch_decode_generic(const DecodeArgs& a, int act_dtype, int cache_
 // ---------------------------------------------------------------------------
 
 // One CTA per (sequence b, chunk of 16 latent columns); thread = head.  Reads
-// o_part[b][s][c][h] (coalesced over heads), merges the splits with weights
+// o_part[b][s][c/4][h][c%4] as float4 (coalesced over heads), merges the splits with weights
 // exp(lse_s - lse), transposes through shared memory and writes o_lat[b][h][c]
 // rows of 16 contiguous columns.  16 columns per thread keep the register count
 // low enough for several CTAs per SM and many loads in flight.
@@ -432,17 +433,25 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
     const float inv_z = z > 0.f ? 1.f / z : 0.f;
     if (blockIdx.y == 0 && a.lse != nullptr)
       a.lse[static_cast<long>(b) * H + h] = z > 0.f ? m + __logf(z) : -INFINITY;
-    const float* op = a.o_part + (static_cast<long>(b) * S * a.d_c + c0) * H + h;
+    const float4* op = reinterpret_cast<const float4*>(a.o_part) +
+                       (static_cast<long>(b) * S * a.d_c + c0) / 4 * H + h;
     float acc[kCombCols];
 #pragma unroll
     for (int c = 0; c < kCombCols; ++c) acc[c] = 0.f;
-    const int nc = min(kCombCols, a.d_c - c0);
+    const int nq = min(kCombCols, a.d_c - c0) / 4;    // d_c is a multiple of 4
     for (int s = 0; s < S; ++s) {
       const float w = cw[s * H + h];
-      const float* os = op + static_cast<long>(s) * a.d_c * H;
+      const float4* os = op + static_cast<long>(s) * (a.d_c / 4) * H;
 #pragma unroll
-      for (int c = 0; c < kCombCols; ++c)
-        if (c < nc) acc[c] += w * os[c * H];
+      for (int g = 0; g < kCombCols / 4; ++g) {
+        if (g < nq) {
+          const float4 v = os[g * H];
+          acc[4 * g] += w * v.x;
+          acc[4 * g + 1] += w * v.y;
+          acc[4 * g + 2] += w * v.z;
+          acc[4 * g + 3] += w * v.w;
+        }
+      }
     }
 #pragma unroll
     for (int c = 0; c < kCombCols; ++c) tile[c][h] = acc[c] * inv_z;

@@ -2,6 +2,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstring>
 #include <map>
 #include <mutex>
 
@@ -56,33 +57,55 @@ bool umma_decode_supported(const mla_ctx* h) {
   const mla_config_t& c = h->cfg;
   return h->cc_major == 10 && c.num_heads == dec::kH && c.d_c == dec::kDc &&
          c.d_c + c.d_r == dec::kD && c.block_size == dec::kTok && c.act_dtype == MLA_BF16 &&
-         c.cache_dtype == MLA_BF16 && encode_fn() != nullptr;
+         (c.cache_dtype == MLA_BF16 || c.cache_dtype == MLA_FP8_E4M3) && encode_fn() != nullptr;
 }
 
+namespace {
+
+template <bool kFp8>
+cudaError_t launch_decode_kernel(const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                 const CUtensorMap& qmap, const DecodeArgs& a, unsigned ctas,
+                                 cudaStream_t s) {
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(dec::decode_umma_kernel<kFp8>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  dec::decode_umma_kernel<kFp8><<<dim3(ctas), dec::threads<kFp8>(), dec::kSmemBytes, s>>>(kmap, vmap, qmap, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_decode_umma(const mla_ctx* h, const DecodeArgs& a, cudaStream_t s) {
+  const bool fp8 = h->cfg.cache_dtype == MLA_FP8_E4M3;
   CUtensorMap kmap, vmap, qmap;
+  std::memset(&kmap, 0, sizeof(kmap));
+  std::memset(&vmap, 0, sizeof(vmap));
   const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * dec::kTok;
-  cudaError_t e = make_map_rows_chunked(&kmap, a.cache, rows, dec::kD * 2, dec::kKBoxes, dec::kTok,
-                                        dec::kKBoxes);
-  if (e != cudaSuccess) return e;
-  e = make_map_rows_chunked(&vmap, a.cache, rows, dec::kD * 2, dec::kKBoxes, dec::kTok, dec::kVBoxes);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (fp8) {
+    // pages and their scales are fetched by untiled bulk copies: 16-byte aligned sources
+    if ((reinterpret_cast<uintptr_t>(a.cache) | reinterpret_cast<uintptr_t>(a.cache_scale)) & 15)
+      return cudaErrorMisalignedAddress;
+  } else {
+    e = make_map_rows_chunked(&kmap, a.cache, rows, dec::kD * 2, dec::kKBoxes, dec::kTok, dec::kKBoxes);
+    if (e != cudaSuccess) return e;
+    e = make_map_rows_chunked(&vmap, a.cache, rows, dec::kD * 2, dec::kKBoxes, dec::kTok, dec::kVBoxes);
+    if (e != cudaSuccess) return e;
+  }
   // absorbed queries as [B*H rows][576 columns], half of a sequence's heads per box
   e = make_map_rows_chunked(&qmap, a.q_lat, static_cast<uint64_t>(a.batch) * dec::kH, dec::kD * 2,
                             dec::kKBoxes, 64, dec::kKBoxes);
   if (e != cudaSuccess) return e;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(dec::decode_umma_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kSmemBytes);
-  });
-  if (attr_err != cudaSuccess) return attr_err;
   const long ctas = 2L * a.batch * a.num_splits;
   if (ctas > 0x7fffffffL) return cudaErrorInvalidValue;
-  dec::decode_umma_kernel<<<dim3(static_cast<unsigned>(ctas)), 256, dec::kSmemBytes, s>>>(kmap, vmap, qmap, a);
-  note_launches(1);
-  return cudaGetLastError();
+  e = fp8 ? launch_decode_kernel<true>(kmap, vmap, qmap, a, static_cast<unsigned>(ctas), s)
+          : launch_decode_kernel<false>(kmap, vmap, qmap, a, static_cast<unsigned>(ctas), s);
+  if (e == cudaSuccess) note_launches(1);
+  return e;
 }
 
 // ---------------------------------------------------------------------------

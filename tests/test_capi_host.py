@@ -112,3 +112,19 @@ def test_binding_counts_pages_from_the_cache_size():
     assert m._num_blocks(h, torch.empty(7, 64, 576, dtype=torch.uint8)) == 7
     with pytest.raises(ValueError):
         m._num_blocks(h, torch.empty(100, 576))
+
+
+def test_binding_checks_the_scale_array_length():
+    """An fp8 cache's scales need one fp32 per cache row: a shorter array would
+    let the kernels read past it, so the binding refuses it before any call."""
+    import types
+
+    import torch
+    h = types.SimpleNamespace(cfg=types.SimpleNamespace(block_size=64, d_c=512, d_r=64))
+    cache = torch.empty(3 * 64, 576, dtype=torch.uint8)
+    assert m._scale_ptr(h, cache, None) is None
+    assert m._scale_ptr(h, cache, torch.empty(3 * 64, dtype=torch.float32)) is not None
+    with pytest.raises(ValueError):
+        m._scale_ptr(h, cache, torch.empty(3 * 64 - 1, dtype=torch.float32))
+    with pytest.raises(ValueError):
+        m._scale_ptr(h, cache, torch.empty(3 * 64, dtype=torch.float64))

@@ -16,10 +16,11 @@ from helpers import assert_close
 pytestmark = pytest.mark.gpu
 
 
-def test_bounded_waits_report_timeout_and_context_survives():
+@pytest.mark.parametrize("name", ["v2_b32_l2048", "v2_b2_l128k_fp8"])
+def test_bounded_waits_report_timeout_and_context_survives(name):
     from mla_latent_kv_19_b200 import mla_last_device_error, mla_set_wait_limit
     from mla_latent_kv_19_b200.step import DecodeStep
-    wl = workloads.make("v2_b32_l2048", batch=2, context=700)
+    wl = workloads.make(name, batch=2, context=700)
     st = DecodeStep(wl, num_splits=2)
     st.append()
     st.absorb()
@@ -34,17 +35,19 @@ def test_bounded_waits_report_timeout_and_context_survives():
     assert mla_last_device_error(st.h) == 0
     g = st.outputs()
     st.close()
-    r = oracle.step_outputs(wl)
+    # an e4m3 cache is compared with the oracle run on its own e4m3 rows
+    r = oracle.step_outputs(wl, fp8_dequant=wl.cache_dtype == "fp8_e4m3")
     for k in ("o_lat", "lse", "y"):
         assert_close(k, g[k], r[k])
 
 
-def test_out_of_range_page_in_decode_is_reported_not_read():
+@pytest.mark.parametrize("name", ["v2_b32_l2048", "v2_b2_l128k_fp8"])
+def test_out_of_range_page_in_decode_is_reported_not_read(name):
     """A page-table entry outside the pool is skipped (masked, read from page 0)
     and reported; the other sequences are unaffected."""
     from mla_latent_kv_19_b200 import mla_last_device_error
     from mla_latent_kv_19_b200.step import DecodeStep
-    wl = workloads.make("v2_b32_l2048", batch=3, context=600)
+    wl = workloads.make(name, batch=3, context=600)
     st = DecodeStep(wl, num_splits=1)
     st.run()
     assert mla_last_device_error(st.h) == 0
@@ -56,6 +59,6 @@ def test_out_of_range_page_in_decode_is_reported_not_read():
     assert mla_last_device_error(st.h) == -6   # MLA_ERR_BAD_INDEX
     g = st.outputs()
     st.close()
-    r = oracle.step_outputs(wl, [0, 2])
+    r = oracle.step_outputs(wl, [0, 2], fp8_dequant=wl.cache_dtype == "fp8_e4m3")
     assert_close("o_lat", g["o_lat"][[0, 2]], r["o_lat"])
     assert np.all(np.isfinite(g["o_lat"][1]))
