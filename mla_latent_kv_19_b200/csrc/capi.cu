@@ -338,7 +338,7 @@ int mla_decode_combine(mla_handle_t h, int32_t batch, int32_t max_seq_len, int32
   a.num_heads = h->cfg.num_heads;
   a.d_c = h->cfg.d_c;
   a.num_splits = S;
-  return map_cuda(launch_combine(a, h->cfg.act_dtype, stream));
+  return map_cuda(launch_combine(a, h->cfg.act_dtype, h->num_sms, stream));
 }
 
 int mla_decode(mla_handle_t h, const void* q_lat, const void* cache, const float* cache_scale,

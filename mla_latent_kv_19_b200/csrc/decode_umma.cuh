@@ -1,6 +1,6 @@
 // Split-KV MLA decode over the paged latent cache on 5th-generation tensor
 // cores (tcgen05 + TMEM + TMA), for the DeepSeek-V2 shape: H = 128 query
-// heads, latent rows of D = d_c + d_r = 512 + 64 bf16 values, 64-token pages.
+// heads, latent rows of D = d_c + d_r = 512 + 64 values, 64-token pages.
 //
 // Method (DeepSeek V2 MLA page, section 2.3): with W_UK absorbed into the
 // query, every head scores s_hj = scale * q_lat_h . row_j over the shared
@@ -10,32 +10,48 @@
 // O += P V (N = 512).
 //
 // Why two CTAs per (sequence, split): the fp32 accumulator O (128 x 512) fills
-// all 512 TMEM columns of an SM, and Q (128 x 576 bf16 = 144 KB) plus a 72 KB
-// page does not leave room for a pipeline in one SM's shared memory.  A
+// all 512 TMEM columns of an SM, and Q (128 x 576 x 2 bytes = 144 KB) plus a
+// 72 KB page does not leave room for a pipeline in one SM's shared memory.  A
 // cluster of two CTAs splits the roles:
 //
-//   CTA 0 ("score"):  a ring of 3 shared-memory slots of 72 KB, each filled
-//     by ONE 3-D TMA request that lands a whole page (64 rows x 576 columns)
-//     as 9 column chunks of [64 rows x 128 bytes] with the 128-byte swizzle
-//     (the UMMA K-major layout); the first two slots carry Q (two halves of
-//     64 heads) into TMEM (columns 0..287, two bf16 per column; Q is then the
-//     A operand of TS-form UMMAs); S = Q K^T (N = 64, one page per MMA) goes
-//     to one of two TMEM buffers (columns 384/448); four softmax warps (one
-//     TMEM lane quadrant each, one head per thread) run the online softmax and
-//     write P (bf16, UMMA K-major swizzled layout) plus the rescale factors
-//     into the page's own slot -- its K data is no longer needed -- and one
-//     thread ships that message to CTA 1 with a single bulk copy (into one of
-//     three P buffers, once P V has finished reading that buffer's previous
-//     message); CTA 1 frees the slot as soon as the message has landed.
+//   CTA 0 ("score"):  a ring of 3 shared-memory slots of 72 KB.  A page
+//     lands as 9 column chunks of [64 rows x 128 bytes] with the 128-byte
+//     swizzle (the UMMA K-major layout), by two 3-D TMA requests: the "tail"
+//     (chunks 3..8, 48 KB) and the "head" (chunks 0..2, 24 KB).  The first two
+//     slots carry Q (two halves of 64 heads) into TMEM (columns 0..287, two
+//     values per column; Q is then the A operand of TS-form UMMAs).
+//     S = Q K^T (N = 64, one page per MMA, tail chunks first) goes to one of
+//     two TMEM buffers (columns 384/448); the commit that reports S also
+//     frees the slot's tail.  Four softmax warps (one TMEM lane quadrant
+//     each, one head per thread) run the online softmax and write P (UMMA
+//     K-major swizzled layout) plus the rescale factors into the slot's head
+//     -- its K data is no longer needed -- and one thread ships that message
+//     to CTA 1 with a single bulk copy (into one of three P buffers, once P V
+//     has finished reading that buffer's previous message).  CTA 1 frees the
+//     head as soon as the message has landed.  So two thirds of a slot turn
+//     over at the pace of the MMAs, and the head, needed last by the next
+//     page's MMAs, has the softmax and the copy to come back.
 //   CTA 1 ("value"):  O accumulates in TMEM columns 0..511; the same pages'
 //     first 512 columns stream through a 2-stage ring, one 64 KB TMA request
 //     per page (an L2 hit after CTA 0's read); P V is issued as two N = 256
 //     SS-form UMMAs per 16-token K step, V being the MN-major B operand.
 //
+// e4m3 cache (kFp8): a page is 36,864 code bytes, fetched by one bulk copy
+// into the upper part of its slot / stage (inside the slot's tail); four
+// converter warps per CTA expand the codes in place to fp16 (exact: an e4m3
+// value has 4 significant bits and its exponent range lies inside fp16's) in
+// the same swizzled layouts, with integer and fp16 arithmetic only.  The
+// contractions then run with fp16 operands (Q is converted once, P is packed
+// as fp16), and the per-token scale enters the softmax: the score of token j
+// is scale_j times the score against its codes, and the P V operand carries
+// p_j * scale_j while the normaliser sums p_j.
+//
 // Measured on B200: issuing a TMA request costs the producer a few hundred
-// cycles (so requests are whole pages), and a tcgen05.mma with M = 128 costs
-// at least ~60 cycles whatever its N up to 128 (so S takes a full page, N = 64,
-// per instruction rather than half pages).
+// cycles (so requests are whole pages), a tcgen05.mma with M = 128 costs at
+// least ~60 cycles whatever its N up to 128 (so S takes a full page, N = 64,
+// per instruction), and the conversion / transcendental pipe is narrow (so
+// the e4m3 codes are expanded with bit operations, leaving that pipe to the
+// softmax's exponentials).
 //
 // The running maximum is only moved when a tile's maximum exceeds it by more
 // than 8 (log2 units), so P stays <= 256 and O needs rescaling (a TMEM read-
@@ -47,6 +63,8 @@
 // drained, TMEM is released and the kernel returns.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "device_common.cuh"
 #include "sm100_ptx.cuh"
 
@@ -54,10 +72,14 @@ namespace mla {
 namespace dec {
 
 constexpr int kH = 128, kDc = 512, kD = 576, kTok = 64;
-constexpr int kBoxBytes = 64 * 128;                    // 64 rows x 64 bf16 (one column chunk)
+constexpr int kBoxBytes = 64 * 128;                    // 64 rows x 64 two-byte values (one column chunk)
 constexpr int kKBoxes = 9, kVBoxes = 8;                // column chunks of a row / of V
 constexpr int kSlotBytes = kKBoxes * kBoxBytes;        // 73728: 9 chunks x 64 rows x 128 B
 constexpr int kChunkInSlot = kBoxBytes;                // 8192
+constexpr int kHeadChunks = 3;                         // chunks 0..2: the head, which carries the P message
+constexpr int kTailChunks = kKBoxes - kHeadChunks;     // chunks 3..8: the tail
+constexpr int kHeadBytes = kHeadChunks * kBoxBytes;    // 24576
+constexpr int kTailBytes = kTailChunks * kBoxBytes;    // 49152
 constexpr int kQLoads = 2;                             // two halves of 64 heads
 constexpr int kSlots = 3;                              // CTA 0 ring
 constexpr int kVStageBytes = kVBoxes * kBoxBytes;      // 65536
@@ -65,14 +87,17 @@ constexpr int kVStages = 2;
 constexpr int kPBytes = kH * kTok * 2;                 // 16384
 constexpr int kPMsgBytes = kPBytes + kH * 4 + 16;      // P + alpha[128] + flag[4] = 16912
 constexpr int kPBufStride = 17 * 1024;                 // keeps every P tile 1024-byte aligned
+static_assert(kPMsgBytes <= kHeadBytes, "the P message fits in a slot's head");
 constexpr int kMaxTablePages = 512;                    // pages of a split kept in shared memory
 constexpr int kPrefetchPages = 4;                      // L2 prefetch distance ahead of the ring's loads
 // e4m3 cache: a page is 64 rows x 576 code bytes, contiguous in the pool, plus
 // 64 fp32 per-token scales
 constexpr int kPageF8Bytes = kTok * kD;                // 36864
-constexpr int kF8InSlot = kSlotBytes - kPageF8Bytes;   // codes land in a slot's upper half
+constexpr int kF8InSlot = kSlotBytes - kPageF8Bytes;   // codes land in a slot's upper half (in its tail)
+static_assert(kF8InSlot >= kHeadBytes, "e4m3 codes land in the tail");
 constexpr int kF8InStage = kVStageBytes - kPageF8Bytes;
 constexpr int kScaleBytes = kTok * 4;
+constexpr int kScaleRing = 6;                          // tile t's scales live in entry t % 6
 constexpr int kF8UnitsK = kPageF8Bytes / 8 / 128;      // 36 eight-code units per converter thread
 constexpr int kF8UnitsV = kTok * kDc / 8 / 128;        // 32 (V: first 512 columns)
 
@@ -81,27 +106,30 @@ constexpr int kOffRing = 0;
 constexpr int kOffTable0 = kSlots * kSlotBytes;        // 221184
 // CTA 1 map
 constexpr int kOffV = 0;
-constexpr int kPBufs = kSlots;                         // message t lives in buffer t % 3
-constexpr int kOffP = kVStages * kVStageBytes;         // 131072: P messages [3]
+constexpr int kPBufs = 3;                              // tile t's P lives in buffer t % 3
+constexpr int kOffP = kVStages * kVStageBytes;         // 131072: P buffers [3]
 constexpr int kOffLfin = kOffP + kPBufs * kPBufStride; // l[128]
 constexpr int kOffTable1 = kOffLfin + kH * 4;
 constexpr int kRegionEnd = kOffTable0 + kMaxTablePages * 4;
 static_assert(kOffTable1 + kMaxTablePages * 4 <= kRegionEnd, "CTA 1 map overlaps the barriers");
 
 enum Bar {
-  kFull = 0, kEmpty = kFull + kSlots,                                     // CTA 0 ring
-  kSFull = kEmpty + kSlots, kSEmpty = kSFull + 2,                        // CTA 0
+  kFullH = 0, kFullT = kFullH + kSlots,                                   // CTA 0 ring: head / tail landed
+  kEmptyH = kFullT + kSlots, kEmptyT = kEmptyH + kSlots,                 //             head / tail free
+  kSFull = kEmptyT + kSlots, kSEmpty = kSFull + 2,                       // CTA 0
   kQReady = kSEmpty + 2, kStg = kQReady + 1,
-  kVFull = kStg + 2, kVEmpty = kVFull + kVStages,                       // CTA 1
-  kPFull = kVEmpty + kVStages, kPVDone = kPFull + kPBufs,
+  kPBufFree = kStg + 2,                                                   // CTA 0: CTA 1's P buffers
+  kScl = kPBufFree + kPBufs,                                              // CTA 0: e4m3 scales ready
+  kCvtLd = kScl + kScaleRing, kCvtDone = kCvtLd + 1,                     // e4m3 converters
+  kVFull = kCvtDone + kSlots, kVEmpty = kVFull + kVStages,               // CTA 1
+  kVCvt = kVEmpty + kVStages,
+  kPFull = kVCvt + kVStages, kPVDone = kPFull + kPBufs,
   kCorrReq = kPVDone + 2, kCorrDone = kCorrReq + 1, kOFull = kCorrDone + 1, kFin = kOFull + 1,
   kDrain = kFin + 1,
-  kCvtLd = kDrain + 1, kCvtDone = kCvtLd + 1, kVCvt = kCvtDone + kSlots,  // e4m3 converters
-  kPBufFree = kVCvt + kVStages,                                          // CTA 0: CTA 1's P buffers
-  kNumBars = kPBufFree + kPBufs
+  kNumBars = kDrain + 1
 };
-constexpr int kOffScale = kRegionEnd;                  // CTA 0: per-token scales [3 slots][64]
-constexpr int kOffBar = kOffScale + kSlots * kScaleBytes;
+constexpr int kOffScale = kRegionEnd;                  // CTA 0: per-token scales [6][64]
+constexpr int kOffBar = kOffScale + kScaleRing * kScaleBytes;
 // misc words: [0] tmem base, [1] abort, [2] corr tile, [3] P messages CTA 0 sent
 // (written by CTA 0 into CTA 1), [4] messages CTA 1 consumed, [5] messages it armed
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -157,18 +185,29 @@ __device__ __forceinline__ int valid_tokens(const Split& s, int page, int t) {
   return page < 0 ? 0 : min(kTok, s.len - (s.p0 + t) * kTok);
 }
 
-// Two e4m3 codes (low byte first) to two bf16 values.  Exact: an e4m3 value has
-// at most 4 significant bits and its exponent range lies inside bf16's.
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
-  const float2 f = __half22float2(__half2(h));
-  const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
-  return *reinterpret_cast<const uint32_t*>(&b);
+// Eight e4m3 codes (low byte first) to eight fp16 values with bit operations
+// and one fp16 multiply per pair.  The fp16 bits (c & 0x7f) << 7 | (c & 0x80) << 8
+// hold exactly value(c) / 256 for every finite code c: the exponent fields of
+// the two formats differ by 8 and an e4m3 subnormal lands on an fp16 subnormal
+// with the same ratio; the product by 256 is exact.  (The two NaN codes, which
+// the append never writes, read as +-480.)
+__device__ __forceinline__ uint4 e4m3x8_to_f16x8(uint2 v) {
+  const __half2 k256 = __float2half2_rn(256.f);
+  auto cvt = [&](uint32_t four, int sel) -> uint32_t {
+    const uint32_t x = __byte_perm(four, 0u, sel);          // two codes in the low bytes of the halves
+    const uint32_t bits = ((x & 0x007f007fu) << 7) | ((x & 0x00800080u) << 8);
+    const __half2 h = __hmul2(*reinterpret_cast<const __half2*>(&bits), k256);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  };
+  return make_uint4(cvt(v.x, 0x4140), cvt(v.x, 0x4342), cvt(v.y, 0x4140), cvt(v.y, 0x4342));
 }
 
-__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 v) {
-  return make_uint4(e4m3x2_to_bf16x2(v.x), e4m3x2_to_bf16x2(v.x >> 16), e4m3x2_to_bf16x2(v.y),
-                    e4m3x2_to_bf16x2(v.y >> 16));
+// Two bf16 values (one word) to two fp16 values: the absorbed query of an e4m3
+// decode enters the fp16 contraction.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xffff0000u);
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // Threads per CTA: 8 warps, plus 4 converter warps with an e4m3 cache.
@@ -177,8 +216,9 @@ constexpr int threads() { return kFp8 ? 384 : 256; }
 
 template <bool kFp8>
 __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
-    decode_umma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
-                       const __grid_constant__ CUtensorMap qmap, const DecodeArgs a) {
+    decode_umma_kernel(const __grid_constant__ CUtensorMap kmap_h, const __grid_constant__ CUtensorMap kmap_t,
+                       const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap,
+                       const DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -220,8 +260,11 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSlots; ++i) {
-      ptx::mbar_init(bar(kFull + i), 1);
-      ptx::mbar_init(bar(kEmpty + i), 1);
+      ptx::mbar_init(bar(kFullH + i), 1);
+      ptx::mbar_init(bar(kFullT + i), 1);
+      ptx::mbar_init(bar(kEmptyH + i), 1);
+      ptx::mbar_init(bar(kEmptyT + i), 1);
+      ptx::mbar_init(bar(kCvtDone + i), 128);
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(bar(kSFull + i), 1);
@@ -229,11 +272,16 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
       ptx::mbar_init(bar(kPVDone + i), 1);
       ptx::mbar_init(bar(kStg + i), 128);
     }
-    for (int i = 0; i < kPBufs; ++i) ptx::mbar_init(bar(kPFull + i), 1);
+    for (int i = 0; i < kPBufs; ++i) {
+      ptx::mbar_init(bar(kPFull + i), 1);
+      ptx::mbar_init(bar(kPBufFree + i), 1);
+    }
+    for (int i = 0; i < kScaleRing; ++i) ptx::mbar_init(bar(kScl + i), 128);
     ptx::mbar_init(bar(kQReady), 128);
     for (int i = 0; i < kVStages; ++i) {
       ptx::mbar_init(bar(kVFull + i), 1);
       ptx::mbar_init(bar(kVEmpty + i), 1);
+      ptx::mbar_init(bar(kVCvt + i), 128);
     }
     ptx::mbar_init(bar(kCorrReq), 1);
     ptx::mbar_init(bar(kCorrDone), 128);
@@ -241,9 +289,6 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
     ptx::mbar_init(bar(kFin), 128);
     ptx::mbar_init(bar(kDrain), 1);
     ptx::mbar_init(bar(kCvtLd), 128);
-    for (int i = 0; i < kSlots; ++i) ptx::mbar_init(bar(kCvtDone + i), 128);
-    for (int i = 0; i < kVStages; ++i) ptx::mbar_init(bar(kVCvt + i), 128);
-    for (int i = 0; i < kPBufs; ++i) ptx::mbar_init(bar(kPBufFree + i), 1);
     misc[1] = 0u;
     misc[2] = 0u;
     misc[3] = 0u;
@@ -264,14 +309,18 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
 
   if (rank == 0) {
     // =========================== CTA 0: scores and softmax ===========================
+    // Slot use n = 0, 1 carries Q half n; use n >= 2 carries tile t = n - 2.  Each
+    // barrier of a slot completes once per use, so use n waits for parity
+    // (n / 3) & 1 of the slot's "landed" barriers and for the completion of the
+    // previous use (parity ((n / 3) & 1) ^ 1) of its "free" barriers.
     if (warp == 0) {
       if (lane == 0) {
-        // TMA producer over the ring: 2 halves of Q, then one request per page.  A
-        // page's slot comes back when CTA 1 has consumed the P message in it.
-        if (!kFp8) ptx::prefetch_tmap(&kmap);
+        // TMA producer: the two halves of Q, then every page's tail (chunks 3..8;
+        // an e4m3 page: all its codes and scales), each as soon as the slot's
+        // tail is free.  Pages are also fetched into L2 a few tiles ahead, so
+        // that the slot's own loads are L2 hits.
+        if (!kFp8) ptx::prefetch_tmap(&kmap_t);
         ptx::prefetch_tmap(&qmap);
-        // pages are fetched into L2 a few tiles before their slot frees, so that
-        // the slot's own load is an L2 hit
         auto prefetch_page = [&](int t) {
           if (t >= sp.ntiles) return;
           const long pg = max(page_at(a, sp, table, t), 0);
@@ -287,61 +336,100 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         int issued = 0;
         for (int n = 0; n < total; ++n) {
           const int slot = n % kSlots;
-          if (!wait_remote(bar(kEmpty + slot), ((n / kSlots) & 1) ^ 1)) break;
+          if (!wait_local(bar(kEmptyT + slot), ((n / kSlots) & 1) ^ 1)) break;
           const uint32_t dst = sb + kOffRing + slot * kSlotBytes;
           if (n < kQLoads) {
-            ptx::mbar_arrive_expect_tx(bar(kFull + slot), kSlotBytes);
-            ptx::tma_load_3d(dst, &qmap, bar(kFull + slot), 0, sp.b * kH + 64 * n, 0);
+            ptx::mbar_arrive_expect_tx(bar(kFullH + slot), kSlotBytes);
+            ptx::tma_load_3d(dst, &qmap, bar(kFullH + slot), 0, sp.b * kH + 64 * n, 0);
           } else {
-            const int pg = max(page_at(a, sp, table, n - kQLoads), 0);
-            prefetch_page(n - kQLoads + kPrefetchPages);
+            const int t = n - kQLoads;
+            const int pg = max(page_at(a, sp, table, t), 0);
+            prefetch_page(t + kPrefetchPages);
             if (kFp8) {
-              // the page's codes (contiguous) into the slot's upper half, its scales aside
-              ptx::mbar_arrive_expect_tx(bar(kFull + slot), kPageF8Bytes + kScaleBytes);
+              // the page's codes (contiguous) into the slot's upper half, its scales
+              // into scale-ring entry t % 6
+              ptx::mbar_arrive_expect_tx(bar(kFullT + slot), kPageF8Bytes + kScaleBytes);
               ptx::bulk_load(dst + kF8InSlot, static_cast<const uint8_t*>(a.cache) + static_cast<long>(pg) * kPageF8Bytes,
-                             kPageF8Bytes, bar(kFull + slot));
-              ptx::bulk_load(sb + kOffScale + slot * kScaleBytes, a.cache_scale + static_cast<long>(pg) * kTok,
-                             kScaleBytes, bar(kFull + slot));
+                             kPageF8Bytes, bar(kFullT + slot));
+              ptx::bulk_load(sb + kOffScale + (t % kScaleRing) * kScaleBytes,
+                             a.cache_scale + static_cast<long>(pg) * kTok, kScaleBytes, bar(kFullT + slot));
             } else {
-              ptx::mbar_arrive_expect_tx(bar(kFull + slot), kSlotBytes);
-              ptx::tma_load_3d(dst, &kmap, bar(kFull + slot), 0, pg * kTok, 0);
+              ptx::mbar_arrive_expect_tx(bar(kFullT + slot), kTailBytes);
+              ptx::tma_load_3d(dst + kHeadBytes, &kmap_t, bar(kFullT + slot), 0, pg * kTok, kHeadChunks);
             }
           }
           issued = n + 1;
         }
         for (int n = max(0, issued - kSlots); n < issued; ++n)
-          drain(bar(kFull + n % kSlots), (n / kSlots) & 1);
+          drain(bar((n < kQLoads ? kFullH : kFullT) + n % kSlots), (n < kQLoads ? n / kSlots : (n - kQLoads) / kSlots) & 1);
+      }
+      __syncwarp();
+    } else if (warp == 2) {
+      // TMA producer of the pages' heads (chunks 0..2), each as soon as the P
+      // message of the slot's previous page has landed in CTA 1 (bf16 cache; an
+      // e4m3 page has no separate head load)
+      if (!kFp8 && lane == 0) {
+        ptx::prefetch_tmap(&kmap_h);
+        int issued = 0;
+        for (int t = 0; t < sp.ntiles; ++t) {
+          const int n = kQLoads + t, slot = n % kSlots;
+          if (!wait_remote(bar(kEmptyH + slot), ((n / kSlots) & 1) ^ 1)) break;
+          const int pg = max(page_at(a, sp, table, t), 0);
+          ptx::mbar_arrive_expect_tx(bar(kFullH + slot), kHeadBytes);
+          ptx::tma_load_3d(sb + kOffRing + slot * kSlotBytes, &kmap_h, bar(kFullH + slot), 0, pg * kTok, 0);
+          issued = t + 1;
+        }
+        for (int t = max(0, issued - kSlots); t < issued; ++t) {
+          const int n = kQLoads + t;
+          drain(bar(kFullH + n % kSlots), (n / kSlots) & 1);
+        }
       }
       __syncwarp();
     } else if (warp == 1) {
-      // MMA issuer: S[i] = Q K^T, A = Q from TMEM, B = page boxes from the ring
+      // MMA issuer: S[i] = Q K^T, A = Q from TMEM, B = page boxes from the ring;
+      // the tail chunks first, then the head
       if (lane == 0) {
-        constexpr uint32_t idS = ptx::idesc_bf16_f32(128, kTok, false, false);
+        constexpr uint32_t idS = ptx::idesc_f16_f32(128, kTok, false, false, kFp8);
         if (wait_local(bar(kQReady), 0)) {
-          for (int n = 0; n < kQLoads; ++n) ptx::mbar_arrive(bar(kEmpty + n));   // Q is in TMEM
+          for (int n = 0; n < kQLoads; ++n) {   // Q is in TMEM: its slots are free
+            ptx::mbar_arrive(bar(kEmptyH + n));
+            ptx::mbar_arrive(bar(kEmptyT + n));
+          }
 #pragma unroll 1
           for (int t = 0; t < sp.ntiles; ++t) {
             const int i = t & 1;
             const int n = kQLoads + t;
             const int slot = n % kSlots;
             if (!wait_local(bar(kSEmpty + i), ((t >> 1) & 1) ^ 1)) break;
-            // the page in bf16: as landed, or once the converters have expanded its codes
+            // the tail as an operand: as landed, or (e4m3) once the converters have
+            // expanded the whole page
             if (!(kFp8 ? wait_local(bar(kCvtDone + slot), (t / kSlots) & 1)
-                       : wait_local(bar(kFull + slot), (n / kSlots) & 1)))
+                       : wait_local(bar(kFullT + slot), (t / kSlots) & 1)))
               break;
             ptx::tc_fence_after();
             // S[i] = Q K^T over the 9 chunks of K = 576, one page (N = 64) per MMA
             const uint32_t d = tmem + kColS + 64u * i;
             const uint32_t kb = sb + kOffRing + slot * kSlotBytes;
-#pragma unroll 3
-            for (int c = 0; c < kKBoxes; ++c) {
+#pragma unroll 2
+            for (int c = kHeadChunks; c < kKBoxes; ++c) {
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 const uint64_t bd = ptx::sdesc_sw128(kb + c * kChunkInSlot + j * 32, 16, 1024);
-                ptx::umma_ts(d, tmem + kColQ + 32u * c + 8u * j, bd, idS, (c | j) ? 1u : 0u);
+                ptx::umma_ts(d, tmem + kColQ + 32u * c + 8u * j, bd, idS, (c != kHeadChunks || j) ? 1u : 0u);
+              }
+            }
+            if (!kFp8 && !wait_local(bar(kFullH + slot), (n / kSlots) & 1)) break;
+            ptx::tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < kHeadChunks; ++c) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint64_t bd = ptx::sdesc_sw128(kb + c * kChunkInSlot + j * 32, 16, 1024);
+                ptx::umma_ts(d, tmem + kColQ + 32u * c + 8u * j, bd, idS, 1u);
               }
             }
             ptx::umma_commit(bar(kSFull + i));
+            ptx::umma_commit(bar(kEmptyT + slot));   // the tail has been read: it is free
           }
         }
         ptx::umma_commit(bar(kDrain));
@@ -355,8 +443,8 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
       const uint32_t lb = static_cast<uint32_t>(q * 32) << 16;
       // Q half q/2 (ring slot q/2) holds this warp's 32 heads as 9 column chunks
       // of 64 rows; the MMA warp frees the slots once every thread has arrived
-      // on q_ready
-      bool ok = wait_local(bar(kFull + (q >> 1)), 0);
+      // on q_ready.  An e4m3 decode contracts in fp16: Q is converted here.
+      bool ok = wait_local(bar(kFullH + (q >> 1)), 0);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         const int row = r & 63;
@@ -371,6 +459,10 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
             v[4 * ch + 1] = u.y;
             v[4 * ch + 2] = u.z;
             v[4 * ch + 3] = u.w;
+          }
+          if (kFp8) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = bf16x2_to_f16x2(v[e]);
           }
           ptx::tmem_st32(tmem + lb + kColQ + 32u * c, v);
         }
@@ -399,12 +491,11 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         ptx::tc_fence_before();
         ptx::mbar_arrive(bar(kSEmpty + i));
         const int valid = valid_tokens(sp, page_at(a, sp, table, t), t);
-        const int slot = (kQLoads + t) % kSlots;
         // e4m3 cache: row j is scale_j times its codes, so score j is scale_j times
-        // the score against the codes (the scales came in with the page)
-        const float* scl = reinterpret_cast<const float*>(smem + kOffScale + slot * kScaleBytes);
+        // the score against the codes (the converters pass on the landed scales)
+        const float* scl = reinterpret_cast<const float*>(smem + kOffScale + (t % kScaleRing) * kScaleBytes);
         if (kFp8) {
-          w = wait_local(bar(kFull + slot), ((kQLoads + t) / kSlots) & 1);
+          w = wait_local(bar(kScl + t % kScaleRing), (t / kScaleRing) & 1);
           if (!__all_sync(0xffffffffu, w)) break;
         }
         float x[64];
@@ -429,20 +520,22 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         for (int j = 0; j < 32; ++j) {
           const float p0 = live ? ptx::ex2(x[2 * j] - m_used) : 0.f;
           const float p1 = live ? ptx::ex2(x[2 * j + 1] - m_used) : 0.f;
-          __nv_bfloat162 pb;
           if (kFp8) {
             // the P V operand carries scale_j (V holds the codes); l sums the weights
             psum += p0 + p1;
-            pb = __floats2bfloat162_rn(2 * j < valid ? p0 * scl[2 * j] : 0.f,
-                                       2 * j + 1 < valid ? p1 * scl[2 * j + 1] : 0.f);
+            const __half2 ph = __floats2half2_rn(2 * j < valid ? p0 * scl[2 * j] : 0.f,
+                                                 2 * j + 1 < valid ? p1 * scl[2 * j + 1] : 0.f);
+            pk[j] = *reinterpret_cast<const uint32_t*>(&ph);
           } else {
-            pb = __floats2bfloat162_rn(p0, p1);
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
             psum += __low2float(pb) + __high2float(pb);
+            pk[j] = *reinterpret_cast<const uint32_t*>(&pb);
           }
-          pk[j] = *reinterpret_cast<const uint32_t*>(&pb);
         }
         l = l * alpha + psum;
-        // the message goes into this page's ring slot: S(t) has consumed its K data
+        // the message goes into the head of this page's slot: S(t) has consumed
+        // its K data, and CTA 1 frees the head once the message has landed
+        const int slot = (kQLoads + t) % kSlots;
         uint8_t* msg = smem + kOffRing + slot * kSlotBytes;
         uint8_t* prow = msg + r * 128;
 #pragma unroll
@@ -472,16 +565,18 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
       ptx::mbar_arrive_remote(rFin);
       if (r == 0) ptx::st_cluster_u32(ptx::mapa(sb + kOffMisc + 12, 1), sent);
     } else if (kFp8 && warp >= 8) {
-      // converters: expand a landed page's e4m3 codes, in place, into the bf16
-      // chunk-major swizzled layout S = Q K^T reads.  Every thread holds its
-      // share of the codes in registers before any thread writes (the bf16 page
-      // covers the codes' bytes).
+      // converters: expand a landed page's e4m3 codes, in place, into the fp16
+      // chunk-major swizzled layout S = Q K^T reads, and pass the page's scales on
+      // to the softmax.  Every thread holds its share of the codes in registers
+      // before any thread writes (the fp16 page covers the codes' bytes), and the
+      // head is written only once the previous page's P message has left it.
       const int ct = static_cast<int>(threadIdx.x) - 256;
 #pragma unroll 1
       for (int t = 0; t < sp.ntiles; ++t) {
         const int n = kQLoads + t, slot = n % kSlots;
-        bool ok = wait_local(bar(kFull + slot), (n / kSlots) & 1);
+        bool ok = wait_local(bar(kFullT + slot), (t / kSlots) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
+        ptx::mbar_arrive(bar(kScl + t % kScaleRing));
         uint8_t* page = smem + kOffRing + slot * kSlotBytes;
         uint2 u[kF8UnitsK];
 #pragma unroll
@@ -489,12 +584,13 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
           u[k] = *reinterpret_cast<const uint2*>(page + kF8InSlot + (k * 128 + ct) * 8);
         ptx::mbar_arrive(bar(kCvtLd));
         ok = wait_local(bar(kCvtLd), t & 1);
+        ok = ok && wait_remote(bar(kEmptyH + slot), ((n / kSlots) & 1) ^ 1);
         if (!__all_sync(0xffffffffu, ok)) break;
 #pragma unroll
         for (int k = 0; k < kF8UnitsK; ++k) {
           const int g = k * 128 + ct, row = g / 72, cu = g - row * 72;
           *reinterpret_cast<uint4*>(page + (cu >> 3) * kChunkInSlot + row * 128 + (((cu & 7) ^ (row & 7)) << 4)) =
-              e4m3x8_to_bf16x8(u[k]);
+              e4m3x8_to_f16x8(u[k]);
         }
         ptx::fence_proxy_async_cta();              // generic writes -> tensor-core reads
         ptx::mbar_arrive(bar(kCvtDone + slot));
@@ -528,7 +624,7 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
       __syncwarp();
     } else if (warp == 1) {
       // MMA issuer: O += P V  (A = P, K-major; B = V, MN-major; two N = 256 halves)
-      constexpr uint32_t idPV = ptx::idesc_bf16_f32(128, 256, false, true);
+      constexpr uint32_t idPV = ptx::idesc_f16_f32(128, 256, false, true, kFp8);
       int ncorr = 0;
 #pragma unroll 1
       for (int t = 0; t < sp.ntiles; ++t) {
@@ -601,16 +697,16 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
       __syncwarp();
     } else if (warp == 3) {
       // P receiver: arms each message's barrier, waits for the message to land and
-      // at once returns CTA 0's ring slot that carried it
+      // at once returns the head of CTA 0's slot that carried it
       if (lane == 0) {
-        const uint32_t rEmpty = ptx::mapa(bar(kEmpty), 0);
+        const uint32_t rEmptyH = ptx::mapa(bar(kEmptyH), 0);
         for (int t = 0; t < sp.ntiles; ++t) {
           const int pbi = t % kPBufs;
           ptx::mbar_arrive_expect_tx(bar(kPFull + pbi), kPMsgBytes);
           misc[5] = static_cast<uint32_t>(t + 1);
           if (!wait_remote(bar(kPFull + pbi), (t / kPBufs) & 1)) break;
           misc[4] = static_cast<uint32_t>(t + 1);
-          ptx::mbar_arrive_remote(rEmpty + 8u * ((kQLoads + t) % kSlots));
+          ptx::mbar_arrive_remote(rEmptyH + 8u * ((kQLoads + t) % kSlots));
         }
       }
       __syncwarp();
@@ -675,7 +771,7 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         ptx::tc_fence_before();
       }
     } else if (kFp8 && warp >= 8) {
-      // converters: the first 512 columns of a landed page to bf16, in place, in
+      // converters: the first 512 columns of a landed page to fp16, in place, in
       // the stage's chunk-major swizzled layout (the MN-major V operand); rows past
       // the sequence end become zeros so that P = 0 meets finite V
       const int ct = static_cast<int>(threadIdx.x) - 256;
@@ -700,7 +796,7 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         for (int k = 0; k < kF8UnitsV; ++k) {
           const int g = k * 128 + ct, row = g >> 6, cu = g & 63;
           *reinterpret_cast<uint4*>(stage + (cu >> 3) * kBoxBytes + row * 128 + (((cu & 7) ^ (row & 7)) << 4)) =
-              e4m3x8_to_bf16x8(u[k]);
+              e4m3x8_to_f16x8(u[k]);
         }
         ptx::fence_proxy_async_cta();
         ptx::mbar_arrive(bar(kVCvt + st));

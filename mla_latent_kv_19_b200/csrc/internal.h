@@ -95,7 +95,7 @@ cudaError_t launch_append(const AppendArgs& a, int act_dtype, int cache_dtype, b
 cudaError_t launch_absorb_generic(const AbsorbArgs& a, int act_dtype, cudaStream_t s);
 cudaError_t launch_decode_generic(const DecodeArgs& a, int act_dtype, int cache_dtype,
                                   cudaStream_t s);
-cudaError_t launch_combine(const CombineArgs& a, int act_dtype, cudaStream_t s);
+cudaError_t launch_combine(const CombineArgs& a, int act_dtype, int num_sms, cudaStream_t s);
 cudaError_t launch_out_proj_generic(const OutProjArgs& a, int act_dtype, cudaStream_t s);
 
 }  // namespace mla

@@ -16,36 +16,61 @@ namespace mla {
 
 constexpr int kAppendWarps = 4;
 
-// Writes one token's row from a staged fp32 copy (c_KV then raw k_R) held in
-// shared memory by one warp.  RoPE pairs (i, i + d_r/2).
-template <typename CT>
-__device__ void write_row_warp(const AppendArgs& a, const float* stage, int p, long slot,
-                               int lane) {
-  const int D = a.d_c + a.d_r;
-  const int half = a.d_r / 2;
-  const float2* cs = a.rope_cs + static_cast<long>(p) * half;
-  CT* row = reinterpret_cast<CT*>(a.cache) + slot * D;
-  for (int i = lane; i < a.d_c; i += 32) row[i] = cvt_out<CT>(stage[i]);
-  for (int i = lane; i < half; i += 32) {
-    const float x1 = stage[a.d_c + i], x2 = stage[a.d_c + half + i];
-    const float2 r = cs[i];
-    row[a.d_c + i] = cvt_out<CT>(x1 * r.x - x2 * r.y);
-    row[a.d_c + half + i] = cvt_out<CT>(x2 * r.x + x1 * r.y);
+// Stage n values of type T (a 16-byte-aligned row, n * sizeof(T) a multiple of
+// 16) into shared memory as fp32, with 16-byte loads that are all issued
+// before any is used (a row is one round trip, not one per element).
+template <typename T>
+__device__ __forceinline__ void stage_row(float* stage, const T* src, int n, int lane) {
+  constexpr int kPer = 16 / static_cast<int>(sizeof(T));
+  const int nv = n / kPer;
+  const uint4* v = reinterpret_cast<const uint4*>(src);
+  for (int j0 = lane; j0 < nv; j0 += 4 * 32) {
+    uint4 buf[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (j0 + 32 * u < nv) buf[u] = v[j0 + 32 * u];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (j0 + 32 * u < nv) {
+        const T* e = reinterpret_cast<const T*>(&buf[u]);
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) stage[(j0 + 32 * u) * kPer + q] = ld_f32(e, q);
+      }
+    }
   }
 }
 
-__device__ void write_row_warp_fp8(const AppendArgs& a, float* stage, int p, long slot, int lane) {
-  const int D = a.d_c + a.d_r;
+// Store n fp32 staged values as CT with 16-byte stores (n * sizeof(CT) a
+// multiple of 16, dst 16-byte aligned).
+template <typename CT>
+__device__ __forceinline__ void store_row(CT* dst, const float* stage, int n, int lane) {
+  constexpr int kPer = 16 / static_cast<int>(sizeof(CT));
+  uint4* v = reinterpret_cast<uint4*>(dst);
+  for (int j = lane; j < n / kPer; j += 32) {
+    uint4 w;
+    CT* e = reinterpret_cast<CT*>(&w);
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) e[q] = cvt_out<CT>(stage[j * kPer + q]);
+    v[j] = w;
+  }
+}
+
+// Rotate the staged k_R (after c_KV in `stage`) in place at position p:
+// pairs (i, i + d_r/2).  The first rotation factor of each lane comes in
+// preloaded (r0, for i = lane).
+__device__ __forceinline__ void rope_stage(const AppendArgs& a, float* stage, const float2* cs,
+                                           float2 r0, int lane) {
   const int half = a.d_r / 2;
-  const float2* cs = a.rope_cs + static_cast<long>(p) * half;
-  // rotate k in place (each pair is owned by one lane)
   for (int i = lane; i < half; i += 32) {
     const float x1 = stage[a.d_c + i], x2 = stage[a.d_c + half + i];
-    const float2 r = cs[i];
+    const float2 r = i == lane ? r0 : cs[i];
     stage[a.d_c + i] = x1 * r.x - x2 * r.y;
     stage[a.d_c + half + i] = x2 * r.x + x1 * r.y;
   }
-  __syncwarp();
+}
+
+__device__ void write_row_warp_fp8(const AppendArgs& a, const float* stage, long slot, int lane) {
+  const int D = a.d_c + a.d_r;
   float amax = 0.f;
   for (int i = lane; i < D; i += 32) amax = fmaxf(amax, fabsf(stage[i]));
   amax = warp_max(amax);
@@ -60,22 +85,10 @@ __device__ void write_row_warp_fp8(const AppendArgs& a, float* stage, int p, lon
   if (lane == 0) a.cache_scale[slot] = amax / 448.f;
 }
 
-// Resolve the physical slot of token t; false (and an error report) if the
-// sequence, position or page is out of range.
-__device__ __forceinline__ bool resolve_slot(const AppendArgs& a, int t, int* p_out, long* slot) {
-  const int b = a.seq_idx ? a.seq_idx[t] : t;
-  const int p = a.pos[t];
-  if (b < 0 || b >= a.batch || p < 0 || p >= a.max_position ||
-      p / a.block_size >= a.max_blocks) {
-    return false;
-  }
-  const int page = a.block_table[static_cast<long>(b) * a.max_blocks + p / a.block_size];
-  if (page < 0 || page >= a.num_blocks) return false;
-  *p_out = p;
-  *slot = static_cast<long>(page) * a.block_size + p % a.block_size;
-  return true;
-}
-
+// One warp per token.  Round 1 loads the token's sequence, position and values
+// together; round 2 the page-table entry and the RoPE factors, which depend on
+// them; then the row is rotated, converted and written.  An out-of-range
+// sequence, position or page is reported and the token skipped.
 template <typename T, typename CT, bool kFp8, bool kProject>
 __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(AppendArgs a) {
   extern __shared__ float smem[];
@@ -83,18 +96,14 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(AppendArgs a)
   const int D = a.d_c + a.d_r;
   const int t = blockIdx.x * kAppendWarps + warp;
   if (t >= a.num_tokens) return;
-  int p;
-  long slot;
-  if (!resolve_slot(a, t, &p, &slot)) {
-    if (lane == 0) report_error(a.err, MLA_ERR_BAD_INDEX);
-    return;
-  }
+  const int b = a.seq_idx ? a.seq_idx[t] : t;
+  const int p = a.pos[t];
   float* stage = smem + warp * D;
   if (kProject) {
     // c_kv = W_DKV x, k_raw = W_KR x: one output per warp iteration, lanes over d_model
     float* xs = smem + kAppendWarps * D + warp * a.d_model;
     const T* x = reinterpret_cast<const T*>(a.x) + static_cast<long>(t) * a.d_model;
-    for (int i = lane; i < a.d_model; i += 32) xs[i] = ld_f32(x, i);
+    stage_row(xs, x, a.d_model, lane);
     __syncwarp();
     for (int j = 0; j < D; ++j) {
       const T* w = j < a.d_c ? reinterpret_cast<const T*>(a.w_dkv) + static_cast<long>(j) * a.d_model
@@ -106,16 +115,27 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(AppendArgs a)
       if (lane == 0) stage[j] = acc;
     }
   } else {
-    const T* c = reinterpret_cast<const T*>(a.c_kv) + static_cast<long>(t) * a.d_c;
-    const T* k = reinterpret_cast<const T*>(a.k_r) + static_cast<long>(t) * a.d_r;
-    for (int i = lane; i < a.d_c; i += 32) stage[i] = ld_f32(c, i);
-    for (int i = lane; i < a.d_r; i += 32) stage[a.d_c + i] = ld_f32(k, i);
+    stage_row(stage, reinterpret_cast<const T*>(a.c_kv) + static_cast<long>(t) * a.d_c, a.d_c, lane);
+    stage_row(stage + a.d_c, reinterpret_cast<const T*>(a.k_r) + static_cast<long>(t) * a.d_r, a.d_r, lane);
   }
+  const bool in_range = b >= 0 && b < a.batch && p >= 0 && p < a.max_position &&
+                        p / a.block_size < a.max_blocks;
+  const int page = in_range ? a.block_table[static_cast<long>(b) * a.max_blocks + p / a.block_size] : -1;
+  const int half = a.d_r / 2;
+  const float2* cs = a.rope_cs + static_cast<long>(in_range ? p : 0) * half;
+  const float2 r0 = lane < half ? cs[lane] : make_float2(1.f, 0.f);
+  if (page < 0 || page >= a.num_blocks) {
+    if (lane == 0) report_error(a.err, MLA_ERR_BAD_INDEX);
+    return;
+  }
+  const long slot = static_cast<long>(page) * a.block_size + p % a.block_size;
+  __syncwarp();
+  rope_stage(a, stage, cs, r0, lane);
   __syncwarp();
   if constexpr (kFp8) {
-    write_row_warp_fp8(a, stage, p, slot, lane);
+    write_row_warp_fp8(a, stage, slot, lane);
   } else {
-    write_row_warp<CT>(a, stage, p, slot, lane);
+    store_row(reinterpret_cast<CT*>(a.cache) + slot * D, stage, D, lane);
   }
 }
 
@@ -404,18 +424,17 @@ cudaError_t launch_decode_generic(const DecodeArgs& a, int act_dtype, int cache_
 // split merge by log-sum-exp
 // ---------------------------------------------------------------------------
 
-// One CTA per (sequence b, chunk of 16 latent columns); thread = head.  Reads
-// o_part[b][s][c/4][h][c%4] as float4 (coalesced over heads), merges the splits with weights
-// exp(lse_s - lse), transposes through shared memory and writes o_lat[b][h][c]
-// rows of 16 contiguous columns.  16 columns per thread keep the register count
-// low enough for several CTAs per SM and many loads in flight.
-constexpr int kCombCols = 16;
-
-template <typename T>
+// One CTA per (sequence b, chunk of kCols latent columns); thread = head.
+// Reads o_part[b][s][c/4][h][c%4] as float4 (coalesced over heads), merges the
+// splits with weights exp(lse_s - lse), transposes through shared memory and
+// writes o_lat[b][h][c] rows of kCols contiguous columns.  16 columns per CTA
+// keep the register count low with many loads in flight; small batches take 4
+// (four times the CTAs) so that the GPU stays full.
+template <typename T, int kCols>
 __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
   extern __shared__ float cw[];               // [num_splits][H] weights
-  __shared__ float tile[kCombCols][129];      // [c][h], padded
-  const int b = blockIdx.x, c0 = blockIdx.y * kCombCols;
+  __shared__ float tile[kCols][129];          // [c][h], padded
+  const int b = blockIdx.x, c0 = blockIdx.y * kCols;
   const int S = a.num_splits, H = a.num_heads;
   const int h = threadIdx.x;                  // blockDim.x == 128 >= H
   if (h < H) {
@@ -435,15 +454,16 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
       a.lse[static_cast<long>(b) * H + h] = z > 0.f ? m + __logf(z) : -INFINITY;
     const float4* op = reinterpret_cast<const float4*>(a.o_part) +
                        (static_cast<long>(b) * S * a.d_c + c0) / 4 * H + h;
-    float acc[kCombCols];
+    float acc[kCols];
 #pragma unroll
-    for (int c = 0; c < kCombCols; ++c) acc[c] = 0.f;
-    const int nq = min(kCombCols, a.d_c - c0) / 4;    // d_c is a multiple of 4
+    for (int c = 0; c < kCols; ++c) acc[c] = 0.f;
+    const int nq = min(kCols, a.d_c - c0) / 4;        // d_c is a multiple of 4
+#pragma unroll 2
     for (int s = 0; s < S; ++s) {
       const float w = cw[s * H + h];
       const float4* os = op + static_cast<long>(s) * (a.d_c / 4) * H;
 #pragma unroll
-      for (int g = 0; g < kCombCols / 4; ++g) {
+      for (int g = 0; g < kCols / 4; ++g) {
         if (g < nq) {
           const float4 v = os[g * H];
           acc[4 * g] += w * v.x;
@@ -454,22 +474,22 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
       }
     }
 #pragma unroll
-    for (int c = 0; c < kCombCols; ++c) tile[c][h] = acc[c] * inv_z;
+    for (int c = 0; c < kCols; ++c) tile[c][h] = acc[c] * inv_z;
   }
   __syncthreads();
-  // o_lat[b][hh][c0 + cc]: each half warp writes one head row of 16 columns
+  // o_lat[b][hh][c0 + cc]: each group of kCols threads writes one head row
   T* out = reinterpret_cast<T*>(a.o_lat) + static_cast<long>(b) * H * a.d_c;
-  const int cc = threadIdx.x & 15;
-  for (int hh = threadIdx.x >> 4; hh < H; hh += 8)
+  const int cc = threadIdx.x % kCols;
+  for (int hh = threadIdx.x / kCols; hh < H; hh += 128 / kCols)
     if (c0 + cc < a.d_c) out[static_cast<long>(hh) * a.d_c + c0 + cc] = cvt_out<T>(tile[cc][hh]);
 }
 
-cudaError_t launch_combine(const CombineArgs& a, int act_dtype, cudaStream_t s) {
-  if (a.batch == 0) return cudaSuccess;
-  if (a.num_heads > 128) return cudaErrorInvalidValue;
-  dim3 grid(a.batch, (a.d_c + kCombCols - 1) / kCombCols);
+template <int kCols>
+cudaError_t launch_combine_cols(const CombineArgs& a, int act_dtype, cudaStream_t s) {
+  dim3 grid(a.batch, (a.d_c + kCols - 1) / kCols);
   const size_t smem = sizeof(float) * a.num_splits * a.num_heads;
-  void (*k)(CombineArgs) = act_dtype == MLA_FP32 ? combine_kernel<float> : combine_kernel<__nv_bfloat16>;
+  void (*k)(CombineArgs) =
+      act_dtype == MLA_FP32 ? combine_kernel<float, kCols> : combine_kernel<__nv_bfloat16, kCols>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -477,6 +497,14 @@ cudaError_t launch_combine(const CombineArgs& a, int act_dtype, cudaStream_t s) 
   k<<<grid, 128, smem, s>>>(a);
   note_launches(1);
   return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const CombineArgs& a, int act_dtype, int num_sms, cudaStream_t s) {
+  if (a.batch == 0) return cudaSuccess;
+  if (a.num_heads > 128) return cudaErrorInvalidValue;
+  if (static_cast<long>(a.batch) * ((a.d_c + 15) / 16) >= 2L * num_sms)
+    return launch_combine_cols<16>(a, act_dtype, s);
+  return launch_combine_cols<4>(a, act_dtype, s);
 }
 
 // ---------------------------------------------------------------------------

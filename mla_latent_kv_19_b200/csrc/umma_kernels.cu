@@ -63,9 +63,9 @@ bool umma_decode_supported(const mla_ctx* h) {
 namespace {
 
 template <bool kFp8>
-cudaError_t launch_decode_kernel(const CUtensorMap& kmap, const CUtensorMap& vmap,
-                                 const CUtensorMap& qmap, const DecodeArgs& a, unsigned ctas,
-                                 cudaStream_t s) {
+cudaError_t launch_decode_kernel(const CUtensorMap& kmap_h, const CUtensorMap& kmap_t,
+                                 const CUtensorMap& vmap, const CUtensorMap& qmap, const DecodeArgs& a,
+                                 unsigned ctas, cudaStream_t s) {
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
@@ -73,7 +73,8 @@ cudaError_t launch_decode_kernel(const CUtensorMap& kmap, const CUtensorMap& vma
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  dec::decode_umma_kernel<kFp8><<<dim3(ctas), dec::threads<kFp8>(), dec::kSmemBytes, s>>>(kmap, vmap, qmap, a);
+  dec::decode_umma_kernel<kFp8><<<dim3(ctas), dec::threads<kFp8>(), dec::kSmemBytes, s>>>(kmap_h, kmap_t, vmap,
+                                                                                           qmap, a);
   return cudaGetLastError();
 }
 
@@ -81,8 +82,9 @@ cudaError_t launch_decode_kernel(const CUtensorMap& kmap, const CUtensorMap& vma
 
 cudaError_t launch_decode_umma(const mla_ctx* h, const DecodeArgs& a, cudaStream_t s) {
   const bool fp8 = h->cfg.cache_dtype == MLA_FP8_E4M3;
-  CUtensorMap kmap, vmap, qmap;
-  std::memset(&kmap, 0, sizeof(kmap));
+  CUtensorMap kmap_h, kmap_t, vmap, qmap;
+  std::memset(&kmap_h, 0, sizeof(kmap_h));
+  std::memset(&kmap_t, 0, sizeof(kmap_t));
   std::memset(&vmap, 0, sizeof(vmap));
   const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * dec::kTok;
   cudaError_t e = cudaSuccess;
@@ -91,7 +93,10 @@ cudaError_t launch_decode_umma(const mla_ctx* h, const DecodeArgs& a, cudaStream
     if ((reinterpret_cast<uintptr_t>(a.cache) | reinterpret_cast<uintptr_t>(a.cache_scale)) & 15)
       return cudaErrorMisalignedAddress;
   } else {
-    e = make_map_rows_chunked(&kmap, a.cache, rows, dec::kD * 2, dec::kKBoxes, dec::kTok, dec::kKBoxes);
+    // a page's head (chunks 0..2) and tail (chunks 3..8), one request each
+    e = make_map_rows_chunked(&kmap_h, a.cache, rows, dec::kD * 2, dec::kKBoxes, dec::kTok, dec::kHeadChunks);
+    if (e != cudaSuccess) return e;
+    e = make_map_rows_chunked(&kmap_t, a.cache, rows, dec::kD * 2, dec::kKBoxes, dec::kTok, dec::kTailChunks);
     if (e != cudaSuccess) return e;
     e = make_map_rows_chunked(&vmap, a.cache, rows, dec::kD * 2, dec::kKBoxes, dec::kTok, dec::kVBoxes);
     if (e != cudaSuccess) return e;
@@ -102,8 +107,8 @@ cudaError_t launch_decode_umma(const mla_ctx* h, const DecodeArgs& a, cudaStream
   if (e != cudaSuccess) return e;
   const long ctas = 2L * a.batch * a.num_splits;
   if (ctas > 0x7fffffffL) return cudaErrorInvalidValue;
-  e = fp8 ? launch_decode_kernel<true>(kmap, vmap, qmap, a, static_cast<unsigned>(ctas), s)
-          : launch_decode_kernel<false>(kmap, vmap, qmap, a, static_cast<unsigned>(ctas), s);
+  e = fp8 ? launch_decode_kernel<true>(kmap_h, kmap_t, vmap, qmap, a, static_cast<unsigned>(ctas), s)
+          : launch_decode_kernel<false>(kmap_h, kmap_t, vmap, qmap, a, static_cast<unsigned>(ctas), s);
   if (e == cudaSuccess) note_launches(1);
   return e;
 }
@@ -141,9 +146,19 @@ cudaError_t ensure_smem_limit(K kernel, size_t bytes) {
   return e;
 }
 
+// TMEM columns a CTA of the GEMM allocates (the kernel's own rule): one block of
+// 32/64/128/256 columns per M tile, rounded up to a power of two.
+int gemm_tmem_cols(const gemm::Params& p) {
+  const int ncpt = p.n <= 32 ? 32 : (p.n <= 64 ? 64 : (p.n <= 128 ? 128 : 256));
+  int cols = 32;
+  while (cols < ncpt * p.mt_per_cta) cols <<= 1;
+  return cols;
+}
+
 template <bool kAMn, gemm::Epi kEpi>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tx, gemm::Params p, dim3 grid,
                         cudaStream_t s) {
+  if (gemm_tmem_cols(p) > 512) return cudaErrorInvalidValue;     // TMEM holds 512 columns
   // as many stages as requested that fit in shared memory (larger batches: fewer)
   while (p.stages > 2 && gemm_smem_bytes(p) > 232448) --p.stages;
   const size_t smem = gemm_smem_bytes(p);
@@ -186,7 +201,9 @@ cudaError_t launch_absorb_umma(const mla_ctx* h, const AbsorbArgs& a, cudaStream
   p.k_chunks = a.d_nope / gemm::kKc;
   p.k_split = 1;
   p.m_per_group = a.d_c;
-  p.mt_per_cta = a.d_c / gemm::kM;      // one CTA per head
+  // all M tiles of a head in one CTA while their accumulators fit in TMEM
+  // (4 x 128 columns up to 128 tokens); larger batches take two CTAs per head
+  p.mt_per_cta = n <= 128 ? a.d_c / gemm::kM : a.d_c / gemm::kM / 2;
   p.kcs = 2;
   p.a_row_group = a.d_nope;
   p.x_col_group = a.d_nope;
@@ -203,7 +220,8 @@ cudaError_t launch_absorb_umma(const mla_ctx* h, const AbsorbArgs& a, cudaStream
   p.max_position = a.max_position;
   p.err = a.err;
   p.wait_limit = h->wait_limit;
-  return launch_gemm<true, gemm::Epi::kAbsorb>(ta, tx, p, dim3(H, 1), s);
+  const int ctas_per_head = (a.d_c / gemm::kM) / p.mt_per_cta;
+  return launch_gemm<true, gemm::Epi::kAbsorb>(ta, tx, p, dim3(H * ctas_per_head, 1), s);
 }
 
 bool umma_out_proj_supported(const mla_ctx* h, int batch) {
@@ -250,10 +268,13 @@ cudaError_t launch_out_proj_umma(const mla_ctx* h, const OutProjArgs& a, void* e
   // partial[s][b][m] = sum over this split's K of W_O[m][k] o[b][k]
   float* part = static_cast<float*>(extra);
   {
+    // 64 KB weight boxes in two stages stream faster than smaller boxes in more
+    // stages (measured); larger batches fall back to 32 KB boxes to fit
+    const int kcs = 2 * (gemm::kM + n) * gemm::kKc * 2 * 4 + 4096 <= 232448 ? 4 : 2;
     CUtensorMap ta, tx;
-    cudaError_t e = make_map_rows_chunked(&ta, a.w_o, a.d_model, kdim * 2, kdim / gemm::kKc, gemm::kM, 2);
+    cudaError_t e = make_map_rows_chunked(&ta, a.w_o, a.d_model, kdim * 2, kdim / gemm::kKc, gemm::kM, kcs);
     if (e != cudaSuccess) return e;
-    e = make_map_rows_chunked(&tx, a.o, a.batch, kdim * 2, kdim / gemm::kKc, n, 2);
+    e = make_map_rows_chunked(&tx, a.o, a.batch, kdim * 2, kdim / gemm::kKc, n, kcs);
     if (e != cudaSuccess) return e;
     gemm::Params p{};
     p.n = n;
@@ -262,10 +283,10 @@ cudaError_t launch_out_proj_umma(const mla_ctx* h, const OutProjArgs& a, void* e
     p.k_split = kOProjSplits;
     p.m_per_group = a.d_model;
     p.mt_per_cta = 1;
-    p.kcs = 2;
+    p.kcs = kcs;
     p.a_row_group = 0;
     p.x_col_group = 0;
-    p.stages = 5;
+    p.stages = kcs == 4 ? 2 : 5;
     p.out = part;
     p.out_ld = a.d_model;
     p.out_group = 0;

@@ -1,0 +1,71 @@
+"""GPU parity of the two projection calls at batch sizes that exercise the
+tensor-core GEMM's padding of the batch (the UMMA N dimension, a multiple of
+16), its box-depth choice for the W_O stream (deeper boxes for small batches,
+shallower ones from ~96 tokens) and the largest supported batch (256), against
+the fp64 oracle:
+
+* mla_absorb_q:  q~[b,h] = W_UK_h^T q_nope[b,h] (+) RoPE(q_pe[b,h], pos_b)
+  (DeepSeek V2 MLA page, sections 2.2 and 2.3);
+* mla_out_proj:  o[b,h] = W_UV_h o_lat[b,h], y[b] = W_O concat_h o[b,h]
+  (section 2.3, W_UV absorbed into the output side)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from helpers import assert_close
+
+pytestmark = pytest.mark.gpu
+
+BATCHES = [1, 17, 100, 256]
+
+
+def _handle(d):
+    from mla_latent_kv_19_b200 import Handle
+    from mla_latent_kv_19_b200.step import softmax_scale
+    return Handle(num_heads=d["num_heads"], d_c=d["d_c"], d_r=d["d_r"], d_nope=d["d_nope"],
+                  d_v=d["d_v"], d_model=d["d_model"], softmax_scale=softmax_scale(d["d_nope"], d["d_r"]),
+                  max_position=4096)
+
+
+@pytest.mark.parametrize("batch", BATCHES)
+def test_absorb_against_oracle(batch):
+    from mla_latent_kv_19_b200 import mla_absorb_q, mla_last_device_error
+    from mla_latent_kv_19_b200.step import to_device
+    wl = workloads.make("v2_b32_l2048", batch=batch, context=64)
+    d = wl.dims
+    rng = np.random.default_rng(1000 + batch)
+    pos = rng.integers(0, 4096, size=batch).astype(np.int32)
+    h = _handle(d)
+    q_lat = torch.empty(batch, d["num_heads"], d["d_c"] + d["d_r"], dtype=torch.bfloat16, device="cuda")
+    mla_absorb_q(h, to_device(wl.q_nope, "cuda"), to_device(wl.q_pe, "cuda"), to_device(pos, "cuda"),
+                 to_device(wl.w_uk, "cuda"), q_lat)
+    assert mla_last_device_error(h) == 0
+    g = q_lat.float().cpu().numpy()
+    h.close()
+    r = oracle.absorb_q(wl.to_f64(wl.q_nope), wl.to_f64(wl.q_pe), wl.to_f64(wl.w_uk), pos, wl.rope_base)
+    assert_close("q_lat", g, r)
+
+
+@pytest.mark.parametrize("batch", BATCHES)
+def test_out_proj_against_oracle(batch):
+    from mla_latent_kv_19_b200 import mla_last_device_error, mla_out_proj, mla_out_proj_workspace_bytes
+    from mla_latent_kv_19_b200.step import to_device
+    wl = workloads.make("v2_b32_l2048", batch=1, context=64)
+    d = wl.dims
+    rng = np.random.default_rng(2000 + batch)
+    o_lat = workloads.f32_to_bf16_bits(
+        rng.standard_normal((batch, d["num_heads"], d["d_c"])).astype(np.float32))
+    h = _handle(d)
+    ws = torch.empty(max(mla_out_proj_workspace_bytes(h, batch), 256), dtype=torch.uint8, device="cuda")
+    y = torch.empty(batch, d["d_model"], dtype=torch.bfloat16, device="cuda")
+    o = torch.empty(batch, d["num_heads"], d["d_v"], dtype=torch.bfloat16, device="cuda")
+    mla_out_proj(h, to_device(o_lat, "cuda"), to_device(wl.w_uv, "cuda"), to_device(wl.w_o, "cuda"), ws, y, o)
+    assert mla_last_device_error(h) == 0
+    g_y, g_o = y.float().cpu().numpy(), o.float().cpu().numpy()
+    h.close()
+    r_o = oracle.up_project_out(workloads.bf16_to_f64(o_lat), wl.to_f64(wl.w_uv))
+    r_y = oracle.out_project(r_o, wl.to_f64(wl.w_o))
+    assert_close("o", g_o, r_o)
+    assert_close("y", g_y, r_y)
