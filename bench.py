@@ -43,11 +43,19 @@ WORKLOAD_TEXT = {
     "v2_b2_l128k_fp8": "V2 dims, batch 2, context 131072, e4m3 cache with per-token fp32 scale",
 }
 STAGES = ("append", "absorb", "decode_partial", "decode_combine", "out_proj")
+# the sources that define each tensor-core stage's kernel (its device code, the
+# PTX wrappers it uses and its launcher): a traffic figure taken by ncu is only
+# reported while all of them are unchanged
 KERNEL_FILES = {
     "decode_partial": ["mla_latent_kv_19_b200/csrc/decode_umma.cuh",
-                       "mla_latent_kv_19_b200/csrc/kernels_generic.cu"],
+                       "mla_latent_kv_19_b200/csrc/sm100_ptx.cuh",
+                       "mla_latent_kv_19_b200/csrc/umma_kernels.cu"],
     "out_proj": ["mla_latent_kv_19_b200/csrc/gemm_umma.cuh",
-                 "mla_latent_kv_19_b200/csrc/kernels_generic.cu"],
+                 "mla_latent_kv_19_b200/csrc/sm100_ptx.cuh",
+                 "mla_latent_kv_19_b200/csrc/umma_kernels.cu"],
+    "absorb": ["mla_latent_kv_19_b200/csrc/gemm_umma.cuh",
+               "mla_latent_kv_19_b200/csrc/sm100_ptx.cuh",
+               "mla_latent_kv_19_b200/csrc/umma_kernels.cu"],
 }
 
 

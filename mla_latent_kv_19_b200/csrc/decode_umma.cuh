@@ -89,7 +89,7 @@ constexpr int kPMsgBytes = kPBytes + kH * 4 + 16;      // P + alpha[128] + flag[
 constexpr int kPBufStride = 17 * 1024;                 // keeps every P tile 1024-byte aligned
 static_assert(kPMsgBytes <= kHeadBytes, "the P message fits in a slot's head");
 constexpr int kMaxTablePages = 512;                    // pages of a split kept in shared memory
-constexpr int kPrefetchPages = 4;                      // L2 prefetch distance ahead of the ring's loads
+constexpr int kPrefetchPages = 0;                      // L2 prefetch distance ahead of the ring's loads (0: none)
 // e4m3 cache: a page is 64 rows x 576 code bytes, contiguous in the pool, plus
 // 64 fp32 per-token scales
 constexpr int kPageF8Bytes = kTok * kD;                // 36864
@@ -125,8 +125,8 @@ enum Bar {
   kVCvt = kVEmpty + kVStages,
   kPFull = kVCvt + kVStages, kPVDone = kPFull + kPBufs,
   kCorrReq = kPVDone + 2, kCorrDone = kCorrReq + 1, kOFull = kCorrDone + 1, kFin = kOFull + 1,
-  kDrain = kFin + 1,
-  kNumBars = kDrain + 1
+  kDrain = kFin + 1, kDrain2 = kDrain + 1,                               // MMA issuers' drains
+  kNumBars = kDrain2 + 1
 };
 constexpr int kOffScale = kRegionEnd;                  // CTA 0: per-token scales [6][64]
 constexpr int kOffBar = kOffScale + kScaleRing * kScaleBytes;
@@ -288,6 +288,7 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
     ptx::mbar_init(bar(kOFull), 1);
     ptx::mbar_init(bar(kFin), 128);
     ptx::mbar_init(bar(kDrain), 1);
+    ptx::mbar_init(bar(kDrain2), 1);
     ptx::mbar_init(bar(kCvtLd), 128);
     misc[1] = 0u;
     misc[2] = 0u;
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         if (!kFp8) ptx::prefetch_tmap(&kmap_t);
         ptx::prefetch_tmap(&qmap);
         auto prefetch_page = [&](int t) {
-          if (t >= sp.ntiles) return;
+          if (kPrefetchPages == 0 || t >= sp.ntiles) return;
           const long pg = max(page_at(a, sp, table, t), 0);
           if (kFp8) {
             ptx::prefetch_l2(static_cast<const uint8_t*>(a.cache) + pg * kPageF8Bytes, kPageF8Bytes);
@@ -385,18 +386,23 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         }
       }
       __syncwarp();
-    } else if (warp == 1) {
-      // MMA issuer: S[i] = Q K^T, A = Q from TMEM, B = page boxes from the ring;
-      // the tail chunks first, then the head
+    } else if (warp == 1 || warp == 3) {
+      // two MMA issuers, warp 1 for even tiles and warp 3 for odd ones (one S
+      // buffer each): two independent streams of N = 64 MMAs keep the tensor
+      // core about twice as busy as one (measured).  S[i] = Q K^T, A = Q from
+      // TMEM, B = page boxes from the ring; the tail chunks first, then the head.
+      const int w = warp == 1 ? 0 : 1;
       if (lane == 0) {
         constexpr uint32_t idS = ptx::idesc_f16_f32(128, kTok, false, false, kFp8);
         if (wait_local(bar(kQReady), 0)) {
-          for (int n = 0; n < kQLoads; ++n) {   // Q is in TMEM: its slots are free
-            ptx::mbar_arrive(bar(kEmptyH + n));
-            ptx::mbar_arrive(bar(kEmptyT + n));
+          if (w == 0) {
+            for (int n = 0; n < kQLoads; ++n) {   // Q is in TMEM: its slots are free
+              ptx::mbar_arrive(bar(kEmptyH + n));
+              ptx::mbar_arrive(bar(kEmptyT + n));
+            }
           }
 #pragma unroll 1
-          for (int t = 0; t < sp.ntiles; ++t) {
+          for (int t = w; t < sp.ntiles; t += 2) {
             const int i = t & 1;
             const int n = kQLoads + t;
             const int slot = n % kSlots;
@@ -432,8 +438,8 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
             ptx::umma_commit(bar(kEmptyT + slot));   // the tail has been read: it is free
           }
         }
-        ptx::umma_commit(bar(kDrain));
-        drain(bar(kDrain), 0);
+        ptx::umma_commit(bar(w == 0 ? kDrain : kDrain2));
+        drain(bar(w == 0 ? kDrain : kDrain2), 0);
       }
       __syncwarp();
     } else if (warp >= 4 && warp < 8) {

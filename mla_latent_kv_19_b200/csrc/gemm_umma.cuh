@@ -183,22 +183,46 @@ __global__ void __launch_bounds__(256, 1)
     const int m = q * 32 + lane;                       // row of this thread in a tile
     const uint32_t lb = static_cast<uint32_t>(q * 32) << 16;
     if (kEpi == Epi::kAbsorb && mt0 == 0 && split == 0) {
-      // RoPE(q_pe[b][h], pos[b]) -> q_lat[b][h][d_c:], pairs (i, i + d_r/2)
-      const int half = p.d_r / 2;
+      // RoPE(q_pe[b][h], pos[b]) -> q_lat[b][h][d_c:], pairs (i, i + d_r/2).  Each
+      // thread takes up to 8 pairs per round and issues all their loads before
+      // any store: the positions in one round trip, then the rotation factors and
+      // q_pe values that depend on them in a second (a loop that stores between
+      // its loads would pay two round trips per pair).
+      constexpr int kPer = 8;
+      const int half = p.d_r / 2, total = p.batch * half;
       __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
-      for (int idx = m; idx < p.batch * half; idx += 128) {
-        const int b = idx / half, i = idx % half;
-        const int ps = p.pos[b];
-        if (ps < 0 || ps >= p.max_position) {
-          report_error(p.err, MLA_ERR_BAD_INDEX);
-          continue;
+      for (int base = m; base < total; base += 128 * kPer) {
+        int ps[kPer];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+          const int idx = base + 128 * u;
+          ps[u] = idx < total ? __ldg(p.pos + idx / half) : 0;
         }
-        const float2 r = p.rope_cs[static_cast<long>(ps) * half + i];
-        const long qb = (static_cast<long>(b) * p.num_heads + group) * p.d_r;
-        const float x1 = __bfloat162float(p.q_pe[qb + i]), x2 = __bfloat162float(p.q_pe[qb + half + i]);
-        const long ob = b * p.out_ld + group * p.out_group + p.d_c;
-        out[ob + i] = __float2bfloat16_rn(x1 * r.x - x2 * r.y);
-        out[ob + half + i] = __float2bfloat16_rn(x2 * r.x + x1 * r.y);
+        float2 r[kPer];
+        float x1[kPer], x2[kPer];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+          const int idx = base + 128 * u;
+          const int b = idx / half, i = idx % half;
+          const bool ok = idx < total && ps[u] >= 0 && ps[u] < p.max_position;
+          r[u] = ok ? __ldg(p.rope_cs + static_cast<long>(ps[u]) * half + i) : make_float2(0.f, 0.f);
+          const long qb = (static_cast<long>(b) * p.num_heads + group) * p.d_r;
+          x1[u] = ok ? __bfloat162float(p.q_pe[qb + i]) : 0.f;
+          x2[u] = ok ? __bfloat162float(p.q_pe[qb + half + i]) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+          const int idx = base + 128 * u;
+          if (idx >= total) continue;
+          if (ps[u] < 0 || ps[u] >= p.max_position) {
+            report_error(p.err, MLA_ERR_BAD_INDEX);
+            continue;
+          }
+          const int b = idx / half, i = idx % half;
+          const long ob = b * p.out_ld + group * p.out_group + p.d_c;
+          out[ob + i] = __float2bfloat16_rn(x1[u] * r[u].x - x2[u] * r[u].y);
+          out[ob + half + i] = __float2bfloat16_rn(x2[u] * r[u].x + x1[u] * r[u].y);
+        }
       }
     }
     bool ok = wait(done, 0);
