@@ -14,30 +14,28 @@
 // 72 KB page does not leave room for a pipeline in one SM's shared memory.  A
 // cluster of two CTAs splits the roles:
 //
-//   CTA 0 ("score"):  a ring of 3 shared-memory slots of 72 KB.  A page
-//     lands as 9 column chunks of [64 rows x 128 bytes] with the 128-byte
-//     swizzle (the UMMA K-major layout), by two 3-D TMA requests: the "tail"
-//     (chunks 3..8, 48 KB) and the "head" (chunks 0..2, 24 KB).  The first two
-//     slots carry Q (two halves of 64 heads) into TMEM (columns 0..287, two
-//     values per column; Q is then the A operand of TS-form UMMAs).
-//     S = Q K^T (N = 64, one page per MMA, tail chunks first) goes to one of
-//     two TMEM buffers (columns 384/448); the commit that reports S also
-//     frees the slot's tail.  Four softmax warps (one TMEM lane quadrant
-//     each, one head per thread) run the online softmax and write P (UMMA
-//     K-major swizzled layout) plus the rescale factors into the slot's head
-//     -- its K data is no longer needed -- and one thread ships that message
-//     to CTA 1 with a single bulk copy (into one of three P buffers, once P V
-//     has finished reading that buffer's previous message).  CTA 1 frees the
-//     head as soon as the message has landed.  So two thirds of a slot turn
-//     over at the pace of the MMAs, and the head, needed last by the next
-//     page's MMAs, has the softmax and the copy to come back.
+//   CTA 0 ("score"):  a ring of 3 shared-memory slots of 72 KB, each filled
+//     by ONE 3-D TMA request that lands a whole page (64 rows x 576 columns)
+//     as 9 column chunks of [64 rows x 128 bytes] with the 128-byte swizzle
+//     (the UMMA K-major layout); the first two slots carry Q (two halves of
+//     64 heads) into TMEM (columns 0..287, two values per column; Q is then
+//     the A operand of TS-form UMMAs).  Two MMA warps, for even and odd tiles,
+//     compute S = Q K^T (N = 64, one page per MMA) into two TMEM buffers
+//     (columns 384/448); the commit that reports S also frees the page's slot.
+//     Four softmax warps (one TMEM lane quadrant each, one head per thread) run
+//     the online softmax and send their row of P (UMMA K-major swizzled
+//     layout), the rescale factor and the warp's rescale flag to one of three
+//     P buffers in CTA 1 with asynchronous distributed-shared-memory stores
+//     (st.async), whose bytes CTA 1's barrier counts -- once P V has finished
+//     reading that buffer's previous tile.  A slot is thus held only from its
+//     load to the end of its MMAs.
 //   CTA 1 ("value"):  O accumulates in TMEM columns 0..511; the same pages'
 //     first 512 columns stream through a 2-stage ring, one 64 KB TMA request
 //     per page (an L2 hit after CTA 0's read); P V is issued as two N = 256
 //     SS-form UMMAs per 16-token K step, V being the MN-major B operand.
 //
 // e4m3 cache (kFp8): a page is 36,864 code bytes, fetched by one bulk copy
-// into the upper part of its slot / stage (inside the slot's tail); four
+// into the upper half of its slot / the upper part of its stage; four
 // converter warps per CTA expand the codes in place to fp16 (exact: an e4m3
 // value has 4 significant bits and its exponent range lies inside fp16's) in
 // the same swizzled layouts, with integer and fp16 arithmetic only.  The
@@ -47,11 +45,13 @@
 // p_j * scale_j while the normaliser sums p_j.
 //
 // Measured on B200: issuing a TMA request costs the producer a few hundred
-// cycles (so requests are whole pages), a tcgen05.mma with M = 128 costs at
-// least ~60 cycles whatever its N up to 128 (so S takes a full page, N = 64,
-// per instruction), and the conversion / transcendental pipe is narrow (so
-// the e4m3 codes are expanded with bit operations, leaving that pipe to the
-// softmax's exponentials).
+// cycles (so requests are whole pages); a tcgen05.mma with M = 128 costs one
+// issuing thread ~60 cycles whatever its N up to 128, while two threads issuing
+// independent MMAs get through them twice as fast (hence N = 64 per page and
+// two S issuers); a signal between the two CTAs of the cluster takes ~0.6 us
+// (hence no round trip on a slot's way back to the producer); and the
+// conversion / transcendental pipe is narrow (so the e4m3 codes are expanded
+// with bit operations, leaving that pipe to the softmax's exponentials).
 //
 // The running maximum is only moved when a tile's maximum exceeds it by more
 // than 8 (log2 units), so P stays <= 256 and O needs rescaling (a TMEM read-
@@ -76,10 +76,6 @@ constexpr int kBoxBytes = 64 * 128;                    // 64 rows x 64 two-byte 
 constexpr int kKBoxes = 9, kVBoxes = 8;                // column chunks of a row / of V
 constexpr int kSlotBytes = kKBoxes * kBoxBytes;        // 73728: 9 chunks x 64 rows x 128 B
 constexpr int kChunkInSlot = kBoxBytes;                // 8192
-constexpr int kHeadChunks = 3;                         // chunks 0..2: the head, which carries the P message
-constexpr int kTailChunks = kKBoxes - kHeadChunks;     // chunks 3..8: the tail
-constexpr int kHeadBytes = kHeadChunks * kBoxBytes;    // 24576
-constexpr int kTailBytes = kTailChunks * kBoxBytes;    // 49152
 constexpr int kQLoads = 2;                             // two halves of 64 heads
 constexpr int kSlots = 3;                              // CTA 0 ring
 constexpr int kVStageBytes = kVBoxes * kBoxBytes;      // 65536
@@ -87,14 +83,12 @@ constexpr int kVStages = 2;
 constexpr int kPBytes = kH * kTok * 2;                 // 16384
 constexpr int kPMsgBytes = kPBytes + kH * 4 + 16;      // P + alpha[128] + flag[4] = 16912
 constexpr int kPBufStride = 17 * 1024;                 // keeps every P tile 1024-byte aligned
-static_assert(kPMsgBytes <= kHeadBytes, "the P message fits in a slot's head");
 constexpr int kMaxTablePages = 512;                    // pages of a split kept in shared memory
 constexpr int kPrefetchPages = 0;                      // L2 prefetch distance ahead of the ring's loads (0: none)
 // e4m3 cache: a page is 64 rows x 576 code bytes, contiguous in the pool, plus
 // 64 fp32 per-token scales
 constexpr int kPageF8Bytes = kTok * kD;                // 36864
-constexpr int kF8InSlot = kSlotBytes - kPageF8Bytes;   // codes land in a slot's upper half (in its tail)
-static_assert(kF8InSlot >= kHeadBytes, "e4m3 codes land in the tail");
+constexpr int kF8InSlot = kSlotBytes - kPageF8Bytes;   // codes land in a slot's upper half
 constexpr int kF8InStage = kVStageBytes - kPageF8Bytes;
 constexpr int kScaleBytes = kTok * 4;
 constexpr int kScaleRing = 6;                          // tile t's scales live in entry t % 6
@@ -114,11 +108,10 @@ constexpr int kRegionEnd = kOffTable0 + kMaxTablePages * 4;
 static_assert(kOffTable1 + kMaxTablePages * 4 <= kRegionEnd, "CTA 1 map overlaps the barriers");
 
 enum Bar {
-  kFullH = 0, kFullT = kFullH + kSlots,                                   // CTA 0 ring: head / tail landed
-  kEmptyH = kFullT + kSlots, kEmptyT = kEmptyH + kSlots,                 //             head / tail free
-  kSFull = kEmptyT + kSlots, kSEmpty = kSFull + 2,                       // CTA 0
-  kQReady = kSEmpty + 2, kStg = kQReady + 1,
-  kPBufFree = kStg + 2,                                                   // CTA 0: CTA 1's P buffers
+  kFull = 0, kEmpty = kFull + kSlots,                                     // CTA 0 ring
+  kSFull = kEmpty + kSlots, kSEmpty = kSFull + 2,                        // CTA 0
+  kQReady = kSEmpty + 2,
+  kPBufFree = kQReady + 1,                                                // CTA 0: CTA 1's P buffers
   kScl = kPBufFree + kPBufs,                                              // CTA 0: e4m3 scales ready
   kCvtLd = kScl + kScaleRing, kCvtDone = kCvtLd + 1,                     // e4m3 converters
   kVFull = kCvtDone + kSlots, kVEmpty = kVFull + kVStages,               // CTA 1
@@ -216,9 +209,8 @@ constexpr int threads() { return kFp8 ? 384 : 256; }
 
 template <bool kFp8>
 __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
-    decode_umma_kernel(const __grid_constant__ CUtensorMap kmap_h, const __grid_constant__ CUtensorMap kmap_t,
-                       const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap,
-                       const DecodeArgs a) {
+    decode_umma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                       const __grid_constant__ CUtensorMap qmap, const DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -260,17 +252,14 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSlots; ++i) {
-      ptx::mbar_init(bar(kFullH + i), 1);
-      ptx::mbar_init(bar(kFullT + i), 1);
-      ptx::mbar_init(bar(kEmptyH + i), 1);
-      ptx::mbar_init(bar(kEmptyT + i), 1);
+      ptx::mbar_init(bar(kFull + i), 1);
+      ptx::mbar_init(bar(kEmpty + i), 1);
       ptx::mbar_init(bar(kCvtDone + i), 128);
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(bar(kSFull + i), 1);
       ptx::mbar_init(bar(kSEmpty + i), 128);
       ptx::mbar_init(bar(kPVDone + i), 1);
-      ptx::mbar_init(bar(kStg + i), 128);
     }
     for (int i = 0; i < kPBufs; ++i) {
       ptx::mbar_init(bar(kPFull + i), 1);
@@ -310,17 +299,12 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
 
   if (rank == 0) {
     // =========================== CTA 0: scores and softmax ===========================
-    // Slot use n = 0, 1 carries Q half n; use n >= 2 carries tile t = n - 2.  Each
-    // barrier of a slot completes once per use, so use n waits for parity
-    // (n / 3) & 1 of the slot's "landed" barriers and for the completion of the
-    // previous use (parity ((n / 3) & 1) ^ 1) of its "free" barriers.
+    // Slot use n = 0, 1 carries Q half n; use n >= 2 carries tile t = n - 2.
     if (warp == 0) {
       if (lane == 0) {
-        // TMA producer: the two halves of Q, then every page's tail (chunks 3..8;
-        // an e4m3 page: all its codes and scales), each as soon as the slot's
-        // tail is free.  Pages are also fetched into L2 a few tiles ahead, so
-        // that the slot's own loads are L2 hits.
-        if (!kFp8) ptx::prefetch_tmap(&kmap_t);
+        // TMA producer over the ring: 2 halves of Q, then one request per page,
+        // each as soon as the slot is free (its previous page's MMAs are done).
+        if (!kFp8) ptx::prefetch_tmap(&kmap);
         ptx::prefetch_tmap(&qmap);
         auto prefetch_page = [&](int t) {
           if (kPrefetchPages == 0 || t >= sp.ntiles) return;
@@ -337,11 +321,11 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         int issued = 0;
         for (int n = 0; n < total; ++n) {
           const int slot = n % kSlots;
-          if (!wait_local(bar(kEmptyT + slot), ((n / kSlots) & 1) ^ 1)) break;
+          if (!wait_local(bar(kEmpty + slot), ((n / kSlots) & 1) ^ 1)) break;
           const uint32_t dst = sb + kOffRing + slot * kSlotBytes;
           if (n < kQLoads) {
-            ptx::mbar_arrive_expect_tx(bar(kFullH + slot), kSlotBytes);
-            ptx::tma_load_3d(dst, &qmap, bar(kFullH + slot), 0, sp.b * kH + 64 * n, 0);
+            ptx::mbar_arrive_expect_tx(bar(kFull + slot), kSlotBytes);
+            ptx::tma_load_3d(dst, &qmap, bar(kFull + slot), 0, sp.b * kH + 64 * n, 0);
           } else {
             const int t = n - kQLoads;
             const int pg = max(page_at(a, sp, table, t), 0);
@@ -349,93 +333,57 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
             if (kFp8) {
               // the page's codes (contiguous) into the slot's upper half, its scales
               // into scale-ring entry t % 6
-              ptx::mbar_arrive_expect_tx(bar(kFullT + slot), kPageF8Bytes + kScaleBytes);
+              ptx::mbar_arrive_expect_tx(bar(kFull + slot), kPageF8Bytes + kScaleBytes);
               ptx::bulk_load(dst + kF8InSlot, static_cast<const uint8_t*>(a.cache) + static_cast<long>(pg) * kPageF8Bytes,
-                             kPageF8Bytes, bar(kFullT + slot));
+                             kPageF8Bytes, bar(kFull + slot));
               ptx::bulk_load(sb + kOffScale + (t % kScaleRing) * kScaleBytes,
-                             a.cache_scale + static_cast<long>(pg) * kTok, kScaleBytes, bar(kFullT + slot));
+                             a.cache_scale + static_cast<long>(pg) * kTok, kScaleBytes, bar(kFull + slot));
             } else {
-              ptx::mbar_arrive_expect_tx(bar(kFullT + slot), kTailBytes);
-              ptx::tma_load_3d(dst + kHeadBytes, &kmap_t, bar(kFullT + slot), 0, pg * kTok, kHeadChunks);
+              ptx::mbar_arrive_expect_tx(bar(kFull + slot), kSlotBytes);
+              ptx::tma_load_3d(dst, &kmap, bar(kFull + slot), 0, pg * kTok, 0);
             }
           }
           issued = n + 1;
         }
         for (int n = max(0, issued - kSlots); n < issued; ++n)
-          drain(bar((n < kQLoads ? kFullH : kFullT) + n % kSlots), (n < kQLoads ? n / kSlots : (n - kQLoads) / kSlots) & 1);
-      }
-      __syncwarp();
-    } else if (warp == 2) {
-      // TMA producer of the pages' heads (chunks 0..2), each as soon as the P
-      // message of the slot's previous page has landed in CTA 1 (bf16 cache; an
-      // e4m3 page has no separate head load)
-      if (!kFp8 && lane == 0) {
-        ptx::prefetch_tmap(&kmap_h);
-        int issued = 0;
-        for (int t = 0; t < sp.ntiles; ++t) {
-          const int n = kQLoads + t, slot = n % kSlots;
-          if (!wait_remote(bar(kEmptyH + slot), ((n / kSlots) & 1) ^ 1)) break;
-          const int pg = max(page_at(a, sp, table, t), 0);
-          ptx::mbar_arrive_expect_tx(bar(kFullH + slot), kHeadBytes);
-          ptx::tma_load_3d(sb + kOffRing + slot * kSlotBytes, &kmap_h, bar(kFullH + slot), 0, pg * kTok, 0);
-          issued = t + 1;
-        }
-        for (int t = max(0, issued - kSlots); t < issued; ++t) {
-          const int n = kQLoads + t;
-          drain(bar(kFullH + n % kSlots), (n / kSlots) & 1);
-        }
+          drain(bar(kFull + n % kSlots), (n / kSlots) & 1);
       }
       __syncwarp();
     } else if (warp == 1 || warp == 3) {
       // two MMA issuers, warp 1 for even tiles and warp 3 for odd ones (one S
       // buffer each): two independent streams of N = 64 MMAs keep the tensor
       // core about twice as busy as one (measured).  S[i] = Q K^T, A = Q from
-      // TMEM, B = page boxes from the ring; the tail chunks first, then the head.
+      // TMEM, B = the page's chunks in the ring.
       const int w = warp == 1 ? 0 : 1;
       if (lane == 0) {
         constexpr uint32_t idS = ptx::idesc_f16_f32(128, kTok, false, false, kFp8);
         if (wait_local(bar(kQReady), 0)) {
-          if (w == 0) {
-            for (int n = 0; n < kQLoads; ++n) {   // Q is in TMEM: its slots are free
-              ptx::mbar_arrive(bar(kEmptyH + n));
-              ptx::mbar_arrive(bar(kEmptyT + n));
-            }
-          }
+          if (w == 0)
+            for (int n = 0; n < kQLoads; ++n) ptx::mbar_arrive(bar(kEmpty + n));   // Q is in TMEM
 #pragma unroll 1
           for (int t = w; t < sp.ntiles; t += 2) {
             const int i = t & 1;
             const int n = kQLoads + t;
             const int slot = n % kSlots;
             if (!wait_local(bar(kSEmpty + i), ((t >> 1) & 1) ^ 1)) break;
-            // the tail as an operand: as landed, or (e4m3) once the converters have
-            // expanded the whole page
+            // the page as an operand: as landed, or once the converters have expanded its codes
             if (!(kFp8 ? wait_local(bar(kCvtDone + slot), (t / kSlots) & 1)
-                       : wait_local(bar(kFullT + slot), (t / kSlots) & 1)))
+                       : wait_local(bar(kFull + slot), (n / kSlots) & 1)))
               break;
             ptx::tc_fence_after();
             // S[i] = Q K^T over the 9 chunks of K = 576, one page (N = 64) per MMA
             const uint32_t d = tmem + kColS + 64u * i;
             const uint32_t kb = sb + kOffRing + slot * kSlotBytes;
-#pragma unroll 2
-            for (int c = kHeadChunks; c < kKBoxes; ++c) {
+#pragma unroll 3
+            for (int c = 0; c < kKBoxes; ++c) {
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 const uint64_t bd = ptx::sdesc_sw128(kb + c * kChunkInSlot + j * 32, 16, 1024);
-                ptx::umma_ts(d, tmem + kColQ + 32u * c + 8u * j, bd, idS, (c != kHeadChunks || j) ? 1u : 0u);
-              }
-            }
-            if (!kFp8 && !wait_local(bar(kFullH + slot), (n / kSlots) & 1)) break;
-            ptx::tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < kHeadChunks; ++c) {
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const uint64_t bd = ptx::sdesc_sw128(kb + c * kChunkInSlot + j * 32, 16, 1024);
-                ptx::umma_ts(d, tmem + kColQ + 32u * c + 8u * j, bd, idS, 1u);
+                ptx::umma_ts(d, tmem + kColQ + 32u * c + 8u * j, bd, idS, (c | j) ? 1u : 0u);
               }
             }
             ptx::umma_commit(bar(kSFull + i));
-            ptx::umma_commit(bar(kEmptyT + slot));   // the tail has been read: it is free
+            ptx::umma_commit(bar(kEmpty + slot));   // the page has been read: its slot is free
           }
         }
         ptx::umma_commit(bar(w == 0 ? kDrain : kDrain2));
@@ -450,7 +398,7 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
       // Q half q/2 (ring slot q/2) holds this warp's 32 heads as 9 column chunks
       // of 64 rows; the MMA warp frees the slots once every thread has arrived
       // on q_ready.  An e4m3 decode contracts in fp16: Q is converted here.
-      bool ok = wait_local(bar(kFullH + (q >> 1)), 0);
+      bool ok = wait_local(bar(kFull + (q >> 1)), 0);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         const int row = r & 63;
@@ -477,7 +425,7 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar(kQReady));
 
-      const uint32_t rP = ptx::mapa(sb + kOffP, 1);
+      const uint32_t rP = ptx::mapa(sb + kOffP, 1);    // CTA 1's P buffers
       const uint32_t rL = ptx::mapa(sb + kOffLfin, 1);
       const uint32_t rPFull = ptx::mapa(bar(kPFull), 1);
       const uint32_t rFin = ptx::mapa(bar(kFin), 1);
@@ -504,65 +452,92 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
           w = wait_local(bar(kScl + t % kScaleRing), (t / kScaleRing) & 1);
           if (!__all_sync(0xffffffffu, w)) break;
         }
-        float x[64];
-        float m_tile = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float f0 = kFp8 ? sl2 * scl[j] : sl2, f1 = kFp8 ? sl2 * scl[j + 32] : sl2;
-          x[j] = j < valid ? __uint_as_float(s0[j]) * f0 : -INFINITY;
-          x[j + 32] = j + 32 < valid ? __uint_as_float(s1[j]) * f1 : -INFINITY;
-          m_tile = fmaxf(m_tile, fmaxf(x[j], x[j + 32]));
-        }
-        const bool resc = m_tile > m_used + kRescaleThreshold;
-        float alpha = 1.f;
-        if (resc) {
-          alpha = (m_used == -INFINITY) ? 0.f : ptx::ex2(m_used - m_tile);
-          m_used = m_tile;
-        }
         uint32_t pk[32];
         float psum = 0.f;
-        const bool live = m_used != -INFINITY;
+        float alpha = 1.f;
+        bool resc = false;
+        if constexpr (!kFp8) {
+          // tile max on the raw scores (the scale is positive), then one FFMA per
+          // exponent: p_j = 2^(s_j * scale * log2(e) - m); masking only on a ragged tile
+          if (valid < kTok) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float p0 = live ? ptx::ex2(x[2 * j] - m_used) : 0.f;
-          const float p1 = live ? ptx::ex2(x[2 * j + 1] - m_used) : 0.f;
-          if (kFp8) {
+            for (int j = 0; j < 32; ++j) {
+              if (j >= valid) s0[j] = __float_as_uint(-INFINITY);
+              if (j + 32 >= valid) s1[j] = __float_as_uint(-INFINITY);
+            }
+          }
+          float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            mx[j & 3] = fmaxf(mx[j & 3], fmaxf(__uint_as_float(s0[j]), __uint_as_float(s1[j])));
+          const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+          resc = m_tile > m_used + kRescaleThreshold;
+          if (resc) {
+            alpha = (m_used == -INFINITY) ? 0.f : ptx::ex2(m_used - m_tile);
+            m_used = m_tile;
+          }
+          if (m_used != -INFINITY) {
+            const float nm = -m_used;
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float p0 = ptx::ex2(fmaf(__uint_as_float(s0[2 * j]), sl2, nm));
+              const float p1 = ptx::ex2(fmaf(__uint_as_float(s0[2 * j + 1]), sl2, nm));
+              const float p2 = ptx::ex2(fmaf(__uint_as_float(s1[2 * j]), sl2, nm));
+              const float p3 = ptx::ex2(fmaf(__uint_as_float(s1[2 * j + 1]), sl2, nm));
+              ps[j & 3] += (p0 + p1) + (p2 + p3);
+              const __nv_bfloat162 pa = __floats2bfloat162_rn(p0, p1), pb = __floats2bfloat162_rn(p2, p3);
+              pk[j] = *reinterpret_cast<const uint32_t*>(&pa);
+              pk[j + 16] = *reinterpret_cast<const uint32_t*>(&pb);
+            }
+            psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) pk[j] = 0u;
+          }
+        } else {
+          float x[64];
+          float m_tile = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float f0 = sl2 * scl[j], f1 = sl2 * scl[j + 32];
+            x[j] = j < valid ? __uint_as_float(s0[j]) * f0 : -INFINITY;
+            x[j + 32] = j + 32 < valid ? __uint_as_float(s1[j]) * f1 : -INFINITY;
+            m_tile = fmaxf(m_tile, fmaxf(x[j], x[j + 32]));
+          }
+          resc = m_tile > m_used + kRescaleThreshold;
+          if (resc) {
+            alpha = (m_used == -INFINITY) ? 0.f : ptx::ex2(m_used - m_tile);
+            m_used = m_tile;
+          }
+          const bool live = m_used != -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float p0 = live ? ptx::ex2(x[2 * j] - m_used) : 0.f;
+            const float p1 = live ? ptx::ex2(x[2 * j + 1] - m_used) : 0.f;
             // the P V operand carries scale_j (V holds the codes); l sums the weights
             psum += p0 + p1;
             const __half2 ph = __floats2half2_rn(2 * j < valid ? p0 * scl[2 * j] : 0.f,
                                                  2 * j + 1 < valid ? p1 * scl[2 * j + 1] : 0.f);
             pk[j] = *reinterpret_cast<const uint32_t*>(&ph);
-          } else {
-            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-            psum += __low2float(pb) + __high2float(pb);
-            pk[j] = *reinterpret_cast<const uint32_t*>(&pb);
           }
         }
         l = l * alpha + psum;
-        // the message goes into the head of this page's slot: S(t) has consumed
-        // its K data, and CTA 1 frees the head once the message has landed
-        const int slot = (kQLoads + t) % kSlots;
-        uint8_t* msg = smem + kOffRing + slot * kSlotBytes;
-        uint8_t* prow = msg + r * 128;
+        // row r of P(t), its rescale factor and (lane 0) the warp's rescale flag go
+        // to CTA 1's buffer t % 3 by asynchronous stores counted on its barrier,
+        // once P V(t - 3) has finished reading that buffer
+        w = wait_remote(bar(kPBufFree + t % kPBufs), ((t / kPBufs) & 1) ^ 1);
+        if (!__all_sync(0xffffffffu, w)) break;
+        const uint32_t pbuf = rP + (t % kPBufs) * kPBufStride;
+        const uint32_t pfull = rPFull + 8u * (t % kPBufs);
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        reinterpret_cast<float*>(msg + kPBytes)[r] = alpha;
+          ptx::st_async_v4(pbuf + r * 128 + ((c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                           pk[4 * c + 3], pfull);
+        ptx::st_async_u32(pbuf + kPBytes + r * 4, __float_as_uint(alpha), pfull);
         const unsigned any = __any_sync(0xffffffffu, resc && t > 0);
-        if (lane == 0) reinterpret_cast<uint32_t*>(msg + kPBytes + kH * 4)[q] = any;
-        ptx::fence_proxy_async_cta();              // generic writes -> bulk-copy reads
-        ptx::mbar_arrive(bar(kStg + i));
-        if (r == 0) {
-          // every row of the message is written and CTA 1's buffer t % 3 is no longer
-          // read by P V(t - 3): ship the message in one bulk copy
-          if (wait_local(bar(kStg + i), (t >> 1) & 1) &&
-              wait_remote(bar(kPBufFree + t % kPBufs), ((t / kPBufs) & 1) ^ 1)) {
-            ptx::bulk_copy_to_peer(rP + (t % kPBufs) * kPBufStride, sb + kOffRing + slot * kSlotBytes,
-                                   kPMsgBytes, rPFull + 8u * (t % kPBufs));
-            ++sent;
-          }
-        }
+        if (lane == 0) ptx::st_async_u32(pbuf + kPBytes + kH * 4 + q * 4, any, pfull);
+        if (r == 0) ++sent;
       }
       // this split's log-sum-exp (natural log) and the normaliser for CTA 1
       const long row = (static_cast<long>(sp.b) * a.num_splits + sp.split) * kH + r;
@@ -574,13 +549,12 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
       // converters: expand a landed page's e4m3 codes, in place, into the fp16
       // chunk-major swizzled layout S = Q K^T reads, and pass the page's scales on
       // to the softmax.  Every thread holds its share of the codes in registers
-      // before any thread writes (the fp16 page covers the codes' bytes), and the
-      // head is written only once the previous page's P message has left it.
+      // before any thread writes (the fp16 page covers the codes' bytes).
       const int ct = static_cast<int>(threadIdx.x) - 256;
 #pragma unroll 1
       for (int t = 0; t < sp.ntiles; ++t) {
         const int n = kQLoads + t, slot = n % kSlots;
-        bool ok = wait_local(bar(kFullT + slot), (t / kSlots) & 1);
+        bool ok = wait_local(bar(kFull + slot), (n / kSlots) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
         ptx::mbar_arrive(bar(kScl + t % kScaleRing));
         uint8_t* page = smem + kOffRing + slot * kSlotBytes;
@@ -590,7 +564,6 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
           u[k] = *reinterpret_cast<const uint2*>(page + kF8InSlot + (k * 128 + ct) * 8);
         ptx::mbar_arrive(bar(kCvtLd));
         ok = wait_local(bar(kCvtLd), t & 1);
-        ok = ok && wait_remote(bar(kEmptyH + slot), ((n / kSlots) & 1) ^ 1);
         if (!__all_sync(0xffffffffu, ok)) break;
 #pragma unroll
         for (int k = 0; k < kF8UnitsK; ++k) {
@@ -638,6 +611,7 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         bool ok = wait_local(bar((kFp8 ? kVCvt : kVFull) + st), (t >> 1) & 1);
         ok = ok && wait_remote(bar(kPFull + pbi), (t / kPBufs) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
+        ptx::fence_proxy_async_cta();   // P arrived by asynchronous stores: order it before the MMAs' reads
         const int valid = valid_tokens(sp, page_at(a, sp, table, t), t);
         if (!kFp8 && valid < kTok) {
           // rows past the sequence end: zero them so that P = 0 meets finite V
@@ -690,7 +664,7 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
       __syncwarp();
     } else if (warp == 2) {
       // release: a finished P V frees its V stage and its P buffer (CTA 0 waits
-      // for the latter before shipping the next message into it)
+      // for the latter before sending the next tile's P into it)
       if (lane == 0) {
         const uint32_t rPBufFree = ptx::mapa(bar(kPBufFree), 0);
         for (int t = 0; t < sp.ntiles; ++t) {
@@ -702,17 +676,16 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
       }
       __syncwarp();
     } else if (warp == 3) {
-      // P receiver: arms each message's barrier, waits for the message to land and
-      // at once returns the head of CTA 0's slot that carried it
+      // P receiver: arms each tile's P barrier with the bytes the softmax sends
+      // (16,912) and follows its completion, so that the teardown knows what is
+      // still in flight after a failed wait
       if (lane == 0) {
-        const uint32_t rEmptyH = ptx::mapa(bar(kEmptyH), 0);
         for (int t = 0; t < sp.ntiles; ++t) {
           const int pbi = t % kPBufs;
           ptx::mbar_arrive_expect_tx(bar(kPFull + pbi), kPMsgBytes);
           misc[5] = static_cast<uint32_t>(t + 1);
           if (!wait_remote(bar(kPFull + pbi), (t / kPBufs) & 1)) break;
           misc[4] = static_cast<uint32_t>(t + 1);
-          ptx::mbar_arrive_remote(rEmptyH + 8u * ((kQLoads + t) % kSlots));
         }
       }
       __syncwarp();
@@ -814,7 +787,7 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
   __syncthreads();
   ptx::cluster_sync();       // CTA 1 now sees how many P messages CTA 0 sent
   if (rank == 1 && threadIdx.x == 0) {
-    // after a wait gave up, messages may still be landing: arm and await each one
+    // after a wait gave up, stores may still be landing: arm and await each tile
     // not consumed yet (in order, so that phase parities stay in step)
     const uint32_t sent = misc[3], armed = misc[5];
     for (uint32_t t = misc[4]; t < sent; ++t) {

@@ -41,6 +41,9 @@ struct Params {
   int m_per_group;       // weight rows of one group (head), multiple of 128
   int mt_per_cta;        // M tiles of one group handled by one CTA
   int kcs;               // K chunks per pipeline stage (box depth)
+  int x_chunks;          // > 0: X is loaded once per CTA (all its x_chunks K chunks,
+                         // which must be the CTA's whole K range) and stays resident;
+                         // the stages then carry the weight only
   // A coordinates: K-major: (elem, row = group*a_row_group + m, chunk = k/64)
   //                MN-major: (elem, row = group*a_row_group + k, chunk = m/64)
   int a_row_group;
@@ -80,16 +83,20 @@ __global__ void __launch_bounds__(256, 1)
   const int nst_k = (kc1 - kc0 + p.kcs - 1) / p.kcs;     // stages per M tile
   const int nst = nst_k * p.mt_per_cta;
 
+  const bool xres = p.x_chunks > 0;
   const int a_bytes = kM * kKc * 2 * p.kcs;              // 16 KB per chunk
   const int x_bytes = p.n * kKc * 2 * p.kcs;             // n rows of 128 B per chunk
-  const int stage_bytes = a_bytes + x_bytes;             // multiple of 1024 (n % 8 == 0)
-  const uint32_t bars = sb + p.stages * stage_bytes;
+  const int xres_bytes = xres ? p.n * kKc * 2 * p.x_chunks : 0;
+  const int stage_bytes = a_bytes + (xres ? 0 : x_bytes);  // multiple of 1024 (n % 8 == 0)
+  const uint32_t stage0 = sb + xres_bytes;               // resident X first, then the stages
+  const uint32_t bars = stage0 + p.stages * stage_bytes;
   auto full = [&](int s) { return bars + 8u * s; };
   auto empty = [&](int s) { return bars + 8u * (p.stages + s); };
   const uint32_t done = bars + 8u * (2 * p.stages);
   const uint32_t drainb = done + 8u;
-  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + p.stages * stage_bytes +
-                                                                 8 * (2 * p.stages + 2));
+  const uint32_t xfull = drainb + 8u;
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + xres_bytes + p.stages * stage_bytes +
+                                                                 8 * (2 * p.stages + 3));
   // TMEM: one block of ncpt columns per M tile
   const uint32_t ncpt = p.n <= 32 ? 32u : (p.n <= 64 ? 64u : (p.n <= 128 ? 128u : 256u));
   uint32_t ncols = 32;
@@ -101,12 +108,13 @@ __global__ void __launch_bounds__(256, 1)
     }
     ptx::mbar_init(done, 1);
     ptx::mbar_init(drainb, 1);
+    ptx::mbar_init(xfull, 1);
     misc[1] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncwarp();
   if (warp == 1) {
-    ptx::tmem_alloc(sb + p.stages * stage_bytes + 8 * (2 * p.stages + 2), ncols);
+    ptx::tmem_alloc(ptx::smem_u32(const_cast<uint32_t*>(misc)), ncols);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -129,13 +137,18 @@ __global__ void __launch_bounds__(256, 1)
     if (lane == 0) {
       ptx::prefetch_tmap(&tmA);
       ptx::prefetch_tmap(&tmX);
+      if (xres && nst > 0) {
+        // the CTA's whole slice of X, once
+        ptx::mbar_arrive_expect_tx(xfull, xres_bytes);
+        ptx::tma_load_3d(sb, &tmX, xfull, 0, 0, (group * p.x_col_group) / kKc + kc0);
+      }
       int issued = 0;
       for (int i = 0; i < nst; ++i) {
         const int s = i % p.stages;
         if (!wait(empty(s), ((i / p.stages) & 1) ^ 1)) break;
         const int mt = mt0 + i / nst_k;
         const int kc = kc0 + (i % nst_k) * p.kcs;
-        const uint32_t dA = sb + s * stage_bytes, dX = dA + a_bytes;
+        const uint32_t dA = stage0 + s * stage_bytes, dX = dA + a_bytes;
         ptx::mbar_arrive_expect_tx(full(s), stage_bytes);
         if (kAMn) {
           // rows = K (kcs*64 of them), chunks = two 64-wide slices of this M tile
@@ -143,21 +156,25 @@ __global__ void __launch_bounds__(256, 1)
         } else {
           ptx::tma_load_3d(dA, &tmA, full(s), 0, group * p.a_row_group + mt * kM, kc);
         }
-        ptx::tma_load_3d(dX, &tmX, full(s), 0, 0, (group * p.x_col_group) / kKc + kc);
+        if (!xres) ptx::tma_load_3d(dX, &tmX, full(s), 0, 0, (group * p.x_col_group) / kKc + kc);
         issued = i + 1;
       }
       for (int i = max(0, issued - p.stages); i < issued; ++i)
         ptx::mbar_wait<false>(full(i % p.stages), (i / p.stages) & 1, 0xffffffffu, kWaitNs);
+      if (xres && nst > 0) ptx::mbar_wait<false>(xfull, 0, 0xffffffffu, kWaitNs);
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = ptx::idesc_bf16_f32(kM, p.n, kAMn, false);
-      for (int i = 0; i < nst; ++i) {
+      const bool xok = !xres || nst == 0 || wait(xfull, 0);
+      for (int i = 0; i < nst && xok; ++i) {
         const int s = i % p.stages;
         if (!wait(full(s), (i / p.stages) & 1)) break;
         ptx::tc_fence_after();
-        const uint32_t aB = sb + s * stage_bytes, xB = aB + a_bytes;
+        const uint32_t aB = stage0 + s * stage_bytes;
+        // X chunks of this stage: in the stage, or at their place in the resident slice
+        const uint32_t xB = xres ? sb + ((i % nst_k) * p.kcs) * (p.n * 128) : aB + a_bytes;
         const uint32_t d = tmem + ncpt * static_cast<uint32_t>(i / nst_k);
         const int kin = i % nst_k;
         const int nkc = min(p.kcs, kc1 - (kc0 + kin * p.kcs));   // chunks of this stage in range

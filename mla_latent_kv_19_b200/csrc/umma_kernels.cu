@@ -63,9 +63,8 @@ bool umma_decode_supported(const mla_ctx* h) {
 namespace {
 
 template <bool kFp8>
-cudaError_t launch_decode_kernel(const CUtensorMap& kmap_h, const CUtensorMap& kmap_t,
-                                 const CUtensorMap& vmap, const CUtensorMap& qmap, const DecodeArgs& a,
-                                 unsigned ctas, cudaStream_t s) {
+cudaError_t launch_decode_kernel(const CUtensorMap& kmap, const CUtensorMap& vmap, const CUtensorMap& qmap,
+                                 const DecodeArgs& a, unsigned ctas, cudaStream_t s) {
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
@@ -73,8 +72,7 @@ cudaError_t launch_decode_kernel(const CUtensorMap& kmap_h, const CUtensorMap& k
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  dec::decode_umma_kernel<kFp8><<<dim3(ctas), dec::threads<kFp8>(), dec::kSmemBytes, s>>>(kmap_h, kmap_t, vmap,
-                                                                                           qmap, a);
+  dec::decode_umma_kernel<kFp8><<<dim3(ctas), dec::threads<kFp8>(), dec::kSmemBytes, s>>>(kmap, vmap, qmap, a);
   return cudaGetLastError();
 }
 
@@ -82,9 +80,8 @@ cudaError_t launch_decode_kernel(const CUtensorMap& kmap_h, const CUtensorMap& k
 
 cudaError_t launch_decode_umma(const mla_ctx* h, const DecodeArgs& a, cudaStream_t s) {
   const bool fp8 = h->cfg.cache_dtype == MLA_FP8_E4M3;
-  CUtensorMap kmap_h, kmap_t, vmap, qmap;
-  std::memset(&kmap_h, 0, sizeof(kmap_h));
-  std::memset(&kmap_t, 0, sizeof(kmap_t));
+  CUtensorMap kmap, vmap, qmap;
+  std::memset(&kmap, 0, sizeof(kmap));
   std::memset(&vmap, 0, sizeof(vmap));
   const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * dec::kTok;
   cudaError_t e = cudaSuccess;
@@ -93,10 +90,7 @@ cudaError_t launch_decode_umma(const mla_ctx* h, const DecodeArgs& a, cudaStream
     if ((reinterpret_cast<uintptr_t>(a.cache) | reinterpret_cast<uintptr_t>(a.cache_scale)) & 15)
       return cudaErrorMisalignedAddress;
   } else {
-    // a page's head (chunks 0..2) and tail (chunks 3..8), one request each
-    e = make_map_rows_chunked(&kmap_h, a.cache, rows, dec::kD * 2, dec::kKBoxes, dec::kTok, dec::kHeadChunks);
-    if (e != cudaSuccess) return e;
-    e = make_map_rows_chunked(&kmap_t, a.cache, rows, dec::kD * 2, dec::kKBoxes, dec::kTok, dec::kTailChunks);
+    e = make_map_rows_chunked(&kmap, a.cache, rows, dec::kD * 2, dec::kKBoxes, dec::kTok, dec::kKBoxes);
     if (e != cudaSuccess) return e;
     e = make_map_rows_chunked(&vmap, a.cache, rows, dec::kD * 2, dec::kKBoxes, dec::kTok, dec::kVBoxes);
     if (e != cudaSuccess) return e;
@@ -107,8 +101,8 @@ cudaError_t launch_decode_umma(const mla_ctx* h, const DecodeArgs& a, cudaStream
   if (e != cudaSuccess) return e;
   const long ctas = 2L * a.batch * a.num_splits;
   if (ctas > 0x7fffffffL) return cudaErrorInvalidValue;
-  e = fp8 ? launch_decode_kernel<true>(kmap_h, kmap_t, vmap, qmap, a, static_cast<unsigned>(ctas), s)
-          : launch_decode_kernel<false>(kmap_h, kmap_t, vmap, qmap, a, static_cast<unsigned>(ctas), s);
+  e = fp8 ? launch_decode_kernel<true>(kmap, vmap, qmap, a, static_cast<unsigned>(ctas), s)
+          : launch_decode_kernel<false>(kmap, vmap, qmap, a, static_cast<unsigned>(ctas), s);
   if (e == cudaSuccess) note_launches(1);
   return e;
 }
@@ -124,9 +118,9 @@ constexpr int kOProjSplits = 3;      // K split of W_O: 40 row tiles x 3 = 120 C
 int padded_n(int batch) { return (batch + 15) / 16 * 16; }
 
 size_t gemm_smem_bytes(const gemm::Params& p) {
-  return static_cast<size_t>(p.stages) *
-             (gemm::kM * gemm::kKc * 2 * p.kcs + p.n * gemm::kKc * 2 * p.kcs) +
-         8 * (2 * p.stages + 2) + 16 + 1024;
+  const size_t xres = p.x_chunks > 0 ? static_cast<size_t>(p.n) * gemm::kKc * 2 * p.x_chunks : 0;
+  const size_t stage = gemm::kM * gemm::kKc * 2 * p.kcs + (p.x_chunks > 0 ? 0 : p.n * gemm::kKc * 2 * p.kcs);
+  return xres + static_cast<size_t>(p.stages) * stage + 8 * (2 * p.stages + 3) + 16 + 1024;
 }
 
 // Raise a kernel's dynamic shared-memory limit once (per process) to the
@@ -201,13 +195,14 @@ cudaError_t launch_absorb_umma(const mla_ctx* h, const AbsorbArgs& a, cudaStream
   p.k_chunks = a.d_nope / gemm::kKc;
   p.k_split = 1;
   p.m_per_group = a.d_c;
-  // all M tiles of a head in one CTA while their accumulators fit in TMEM
-  // (4 x 128 columns up to 128 tokens); larger batches take two CTAs per head
-  p.mt_per_cta = n <= 128 ? a.d_c / gemm::kM : a.d_c / gemm::kM / 2;
+  // two M tiles per CTA, two CTAs per head: small CTAs (the head's q_nope slice
+  // loaded once and kept, two 32 KB weight boxes) of which several share an SM
+  p.mt_per_cta = 2;
   p.kcs = 2;
+  p.x_chunks = a.d_nope / gemm::kKc;
   p.a_row_group = a.d_nope;
   p.x_col_group = a.d_nope;
-  p.stages = 4;
+  p.stages = 2;
   p.out = a.q_lat;
   p.out_ld = static_cast<long>(H) * (a.d_c + a.d_r);
   p.out_group = a.d_c + a.d_r;
@@ -237,14 +232,17 @@ cudaError_t launch_out_proj_umma(const mla_ctx* h, const OutProjArgs& a, void* e
                                  cudaStream_t s) {
   const int H = a.num_heads, n = padded_n(a.batch);
   const long kdim = static_cast<long>(H) * a.d_v;
-  // o[b][h][v] = W_UV[h] o_lat[b][h]
+  // o[b][h][v] = W_UV[h] o_lat[b][h]: one CTA per head; while the head's o_lat
+  // slice fits next to two 64 KB weight boxes it is loaded once and kept
   {
+    const bool xres = static_cast<long>(n) * a.d_c * 2 + 2L * gemm::kM * gemm::kKc * 2 * 4 + 4096 <= 232448;
+    const int kcs = xres ? 4 : 2;
     CUtensorMap ta, tx;
     cudaError_t e = make_map_rows_chunked(&ta, a.w_uv, static_cast<uint64_t>(H) * a.d_v, a.d_c * 2,
-                                          a.d_c / gemm::kKc, gemm::kM, 2);
+                                          a.d_c / gemm::kKc, gemm::kM, kcs);
     if (e != cudaSuccess) return e;
     e = make_map_rows_chunked(&tx, a.o_lat, a.batch, static_cast<uint64_t>(H) * a.d_c * 2,
-                              H * a.d_c / gemm::kKc, n, 2);
+                              H * a.d_c / gemm::kKc, n, xres ? a.d_c / gemm::kKc : kcs);
     if (e != cudaSuccess) return e;
     gemm::Params p{};
     p.n = n;
@@ -253,10 +251,11 @@ cudaError_t launch_out_proj_umma(const mla_ctx* h, const OutProjArgs& a, void* e
     p.k_split = 1;
     p.m_per_group = a.d_v;
     p.mt_per_cta = 1;
-    p.kcs = 2;
+    p.kcs = kcs;
+    p.x_chunks = xres ? a.d_c / gemm::kKc : 0;
     p.a_row_group = a.d_v;
     p.x_col_group = a.d_c;
-    p.stages = 4;
+    p.stages = xres ? 2 : 4;
     p.out = a.o;
     p.out_ld = kdim;
     p.out_group = a.d_v;
