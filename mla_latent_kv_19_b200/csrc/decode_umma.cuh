@@ -119,10 +119,12 @@ enum Bar {
   kPFull = kVCvt + kVStages, kPVDone = kPFull + kPBufs,
   kCorrReq = kPVDone + 2, kCorrDone = kCorrReq + 1, kOFull = kCorrDone + 1, kFin = kOFull + 1,
   kDrain = kFin + 1, kDrain2 = kDrain + 1,                               // MMA issuers' drains
-  kNumBars = kDrain2 + 1
+  kStgFull = kDrain2 + 1, kStgFree = kStgFull + 2,                       // CTA 0: bf16 P staging in TMEM
+  kNumBars = kStgFree + 2
 };
 constexpr int kOffScale = kRegionEnd;                  // CTA 0: per-token scales [6][64]
-constexpr int kOffBar = kOffScale + kScaleRing * kScaleBytes;
+constexpr int kOffStg = kOffScale + kScaleRing * kScaleBytes;  // CTA 0: staged alpha [2][128], flags [2][4]
+constexpr int kOffBar = kOffStg + (2 * kH + 8) * 4;
 // misc words: [0] tmem base, [1] abort, [2] corr tile, [3] P messages CTA 0 sent
 // (written by CTA 0 into CTA 1), [4] messages CTA 1 consumed, [5] messages it armed
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -133,6 +135,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQ = 0;                          // CTA 0: Q, 288 columns
 constexpr uint32_t kColS = 384;                        // CTA 0: S[2], 64 columns each
+constexpr uint32_t kColStg = 288;                      // CTA 0 (bf16): staged P[2], 32 columns each
 constexpr uint32_t kColO = 0;                          // CTA 1: O, 512 columns
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -203,9 +206,10 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Threads per CTA: 8 warps, plus 4 converter warps with an e4m3 cache.
+// Threads per CTA: 12 warps.  Warps 8..11 are a second softmax warpgroup with a
+// bf16 cache and the e4m3 converters with an e4m3 cache.
 template <bool kFp8>
-constexpr int threads() { return kFp8 ? 384 : 256; }
+constexpr int threads() { return 384; }
 
 template <bool kFp8>
 __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
@@ -260,20 +264,22 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
       ptx::mbar_init(bar(kSFull + i), 1);
       ptx::mbar_init(bar(kSEmpty + i), 128);
       ptx::mbar_init(bar(kPVDone + i), 1);
+      ptx::mbar_init(bar(kStgFull + i), 128);
+      ptx::mbar_init(bar(kStgFree + i), 128);
     }
     for (int i = 0; i < kPBufs; ++i) {
       ptx::mbar_init(bar(kPFull + i), 1);
       ptx::mbar_init(bar(kPBufFree + i), 1);
     }
     for (int i = 0; i < kScaleRing; ++i) ptx::mbar_init(bar(kScl + i), 128);
-    ptx::mbar_init(bar(kQReady), 128);
+    ptx::mbar_init(bar(kQReady), kFp8 ? 128 : 256);
     for (int i = 0; i < kVStages; ++i) {
       ptx::mbar_init(bar(kVFull + i), 1);
       ptx::mbar_init(bar(kVEmpty + i), 1);
       ptx::mbar_init(bar(kVCvt + i), 128);
     }
     ptx::mbar_init(bar(kCorrReq), 1);
-    ptx::mbar_init(bar(kCorrDone), 128);
+    ptx::mbar_init(bar(kCorrDone), kFp8 ? 128 : 256);
     ptx::mbar_init(bar(kOFull), 1);
     ptx::mbar_init(bar(kFin), 128);
     ptx::mbar_init(bar(kDrain), 1);
@@ -390,6 +396,179 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         drain(bar(w == 0 ? kDrain : kDrain2), 0);
       }
       __syncwarp();
+    } else if (!kFp8 && warp >= 8) {
+      // bf16 cache, senders (one warp per TMEM lane quadrant): help move Q into
+      // TMEM, then for every tile take the P rows the softmax staged in TMEM, with
+      // the rescale factors and flags it staged in shared memory, and send them to
+      // CTA 1's buffer t % 3 by asynchronous stores counted on its barrier, once
+      // P V(t - 3) has read that buffer.  A transfer between the two SMs costs
+      // ~0.8 us per tile this way; here it overlaps the next tile's softmax.
+      const int q = warp & 3;
+      const int r = q * 32 + lane;
+      const uint32_t lb = static_cast<uint32_t>(q * 32) << 16;
+      bool ok = wait_local(bar(kFull + (q >> 1)), 0);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        const int row = r & 63;
+        const uint8_t* base = smem + kOffRing + (q >> 1) * kSlotBytes + row * 128;
+#pragma unroll 1
+        for (int c = 5; c < kKBoxes; ++c) {
+          uint32_t v[32];
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint4 u = *reinterpret_cast<const uint4*>(base + c * kChunkInSlot + ((ch ^ (row & 7)) << 4));
+            v[4 * ch] = u.x;
+            v[4 * ch + 1] = u.y;
+            v[4 * ch + 2] = u.z;
+            v[4 * ch + 3] = u.w;
+          }
+          ptx::tmem_st32(tmem + lb + kColQ + 32u * c, v);
+        }
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar(kQReady));
+
+      const uint32_t rP = ptx::mapa(sb + kOffP, 1);
+      const uint32_t rPFull = ptx::mapa(bar(kPFull), 1);
+      const float* astg = reinterpret_cast<const float*>(smem + kOffStg);
+      const uint32_t* fstg = reinterpret_cast<const uint32_t*>(smem + kOffStg + 2 * kH * 4);
+      uint32_t sent = 0;
+#pragma unroll 1
+      for (int t = 0; t < sp.ntiles && ok; ++t) {
+        const int i = t & 1;
+        bool w = wait_local(bar(kStgFull + i), (t >> 1) & 1);
+        if (!__all_sync(0xffffffffu, w)) break;
+        ptx::tc_fence_after();
+        uint32_t v[32];
+        ptx::tmem_ld32(tmem + lb + kColStg + 32u * i, v);
+        ptx::tmem_wait_ld();
+        const uint32_t alpha = __float_as_uint(astg[i * kH + r]);
+        const uint32_t flag = fstg[i * 4 + q];
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(kStgFree + i));
+        w = wait_remote(bar(kPBufFree + t % kPBufs), ((t / kPBufs) & 1) ^ 1);
+        if (!__all_sync(0xffffffffu, w)) break;
+        const uint32_t pbuf = rP + (t % kPBufs) * kPBufStride;
+        const uint32_t pfull = rPFull + 8u * (t % kPBufs);
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          ptx::st_async_v4(pbuf + r * 128 + ((c ^ (r & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3],
+                           pfull);
+        ptx::st_async_u32(pbuf + kPBytes + r * 4, alpha, pfull);
+        if (lane == 0) ptx::st_async_u32(pbuf + kPBytes + kH * 4 + q * 4, flag, pfull);
+        if (r == 0) ++sent;
+      }
+      if (r == 0) ptx::st_cluster_u32(ptx::mapa(sb + kOffMisc + 12, 1), sent);
+    } else if (!kFp8 && warp >= 4) {
+      // bf16 cache, softmax warpgroup (thread = head row r, TMEM lane quadrant q):
+      // the online softmax of every tile, its P row staged in TMEM and the
+      // rescale factor / flag in shared memory for the senders
+      const int q = warp & 3;
+      const int r = q * 32 + lane;
+      const uint32_t lb = static_cast<uint32_t>(q * 32) << 16;
+      bool ok = wait_local(bar(kFull + (q >> 1)), 0);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        const int row = r & 63;
+        const uint8_t* base = smem + kOffRing + (q >> 1) * kSlotBytes + row * 128;
+#pragma unroll 1
+        for (int c = 0; c < 5; ++c) {
+          uint32_t v[32];
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint4 u = *reinterpret_cast<const uint4*>(base + c * kChunkInSlot + ((ch ^ (row & 7)) << 4));
+            v[4 * ch] = u.x;
+            v[4 * ch + 1] = u.y;
+            v[4 * ch + 2] = u.z;
+            v[4 * ch + 3] = u.w;
+          }
+          ptx::tmem_st32(tmem + lb + kColQ + 32u * c, v);
+        }
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar(kQReady));
+
+      const uint32_t rL = ptx::mapa(sb + kOffLfin, 1);
+      const uint32_t rFin = ptx::mapa(bar(kFin), 1);
+      float* astg = reinterpret_cast<float*>(smem + kOffStg);
+      uint32_t* fstg = reinterpret_cast<uint32_t*>(smem + kOffStg + 2 * kH * 4);
+      const float sl2 = a.scale * kLog2e;
+      float m_used = -INFINITY, l = 0.f;
+#pragma unroll 1
+      for (int t = 0; t < sp.ntiles && ok; ++t) {
+        const int i = t & 1;
+        bool w = wait_local(bar(kSFull + i), (t >> 1) & 1);
+        if (!__all_sync(0xffffffffu, w)) break;
+        ptx::tc_fence_after();
+        uint32_t s0[32], s1[32];
+        ptx::tmem_ld32(tmem + lb + kColS + 64u * i, s0);
+        ptx::tmem_ld32(tmem + lb + kColS + 64u * i + 32u, s1);
+        ptx::tmem_wait_ld();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(kSEmpty + i));
+        const int valid = valid_tokens(sp, page_at(a, sp, table, t), t);
+        // tile max on the raw scores (the scale is positive), then one FFMA per
+        // exponent: p_j = 2^(s_j * scale * log2(e) - m); masking only on a ragged tile
+        if (valid < kTok) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (j >= valid) s0[j] = __float_as_uint(-INFINITY);
+            if (j + 32 >= valid) s1[j] = __float_as_uint(-INFINITY);
+          }
+        }
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          mx[j & 3] = fmaxf(mx[j & 3], fmaxf(__uint_as_float(s0[j]), __uint_as_float(s1[j])));
+        const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+        const bool resc = m_tile > m_used + kRescaleThreshold;
+        float alpha = 1.f;
+        if (resc) {
+          alpha = (m_used == -INFINITY) ? 0.f : ptx::ex2(m_used - m_tile);
+          m_used = m_tile;
+        }
+        uint32_t pk[32];
+        float psum = 0.f;
+        if (m_used != -INFINITY) {
+          const float nm = -m_used;
+          float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float p0 = ptx::ex2(fmaf(__uint_as_float(s0[2 * j]), sl2, nm));
+            const float p1 = ptx::ex2(fmaf(__uint_as_float(s0[2 * j + 1]), sl2, nm));
+            const float p2 = ptx::ex2(fmaf(__uint_as_float(s1[2 * j]), sl2, nm));
+            const float p3 = ptx::ex2(fmaf(__uint_as_float(s1[2 * j + 1]), sl2, nm));
+            ps[j & 3] += (p0 + p1) + (p2 + p3);
+            const __nv_bfloat162 pa = __floats2bfloat162_rn(p0, p1), pb = __floats2bfloat162_rn(p2, p3);
+            pk[j] = *reinterpret_cast<const uint32_t*>(&pa);
+            pk[j + 16] = *reinterpret_cast<const uint32_t*>(&pb);
+          }
+          psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) pk[j] = 0u;
+        }
+        l = l * alpha + psum;
+        // stage: P row in TMEM buffer t & 1, alpha and the warp's rescale flag in
+        // shared memory, once the senders have taken tile t - 2 out of them
+        w = wait_local(bar(kStgFree + i), ((t >> 1) & 1) ^ 1);
+        if (!__all_sync(0xffffffffu, w)) break;
+        ptx::tc_fence_after();
+        ptx::tmem_st32(tmem + lb + kColStg + 32u * i, pk);
+        astg[i * kH + r] = alpha;
+        const unsigned any = __any_sync(0xffffffffu, resc && t > 0);
+        if (lane == 0) fstg[i * 4 + q] = any;
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(kStgFull + i));
+      }
+      // this split's log-sum-exp (natural log) and the normaliser for CTA 1
+      const long row = (static_cast<long>(sp.b) * a.num_splits + sp.split) * kH + r;
+      a.lse_part[row] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+      ptx::st_cluster_u32(rL + r * 4, __float_as_uint(l));
+      ptx::mbar_arrive_remote(rFin);
     } else if (warp >= 4 && warp < 8) {
       // softmax warpgroup: thread = head row r, TMEM lane quadrant q
       const int q = warp & 3;
@@ -689,8 +868,13 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         }
       }
       __syncwarp();
-    } else if (warp >= 4 && warp < 8) {
-      // correction (rescale O rows on request) and epilogue
+    } else if (warp >= 4 && (warp < 8 || !kFp8)) {
+      // correction (rescale O rows on request) and epilogue; with a bf16 cache two
+      // warpgroups share them, warps 4..7 taking O's columns 0..255 and warps 8..11
+      // columns 256..511
+      constexpr int kGroups = kFp8 ? 1 : 2;
+      const int wg = warp >> 3;
+      const int c0 = wg * (16 / kGroups), c1 = c0 + 16 / kGroups;    // 32-column blocks of O
       const int q = warp & 3;
       const int r = q * 32 + lane;
       const uint32_t lb = static_cast<uint32_t>(q * 32) << 16;
@@ -710,7 +894,7 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         const float al =
             reinterpret_cast<const float*>(smem + kOffP + (t % kPBufs) * kPBufStride + kPBytes)[r];
 #pragma unroll 1
-        for (int c = 0; c < 16; ++c) {
+        for (int c = c0; c < c1; ++c) {
           uint32_t v[32];
           ptx::tmem_ld32(tmem + lb + kColO + 32u * c, v);
           ptx::tmem_wait_ld();
@@ -734,10 +918,10 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         const float lsum = reinterpret_cast<const volatile float*>(smem + kOffLfin)[r];
         const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
         if (sp.ntiles == 0) {
-          for (int g = 0; g < kDc / 4; ++g) obase[g * kH] = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int g = 8 * c0; g < 8 * c1; ++g) obase[g * kH] = make_float4(0.f, 0.f, 0.f, 0.f);
         } else {
 #pragma unroll 1
-          for (int c = 0; c < 16; ++c) {
+          for (int c = c0; c < c1; ++c) {
             uint32_t v[32];
             ptx::tmem_ld32(tmem + lb + kColO + 32u * c, v);
             ptx::tmem_wait_ld();
