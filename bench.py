@@ -3,7 +3,8 @@
 
 A step is one pass of the whole path on one batch: append the new token of
 every sequence, absorb the queries, split-KV decode, merge the splits, output
-projection -- five C-ABI calls into libmla.  Default workload: the
+projection -- four C-ABI calls into libmla (the split merge runs inside the
+output projection's first kernel).  Default workload: the
 DeepSeek-V2-shaped decode, batch 32, context 2048, bf16 paged cache.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -42,7 +43,7 @@ WORKLOAD_TEXT = {
     "v2_b4_l32k": "V2 dims, batch 4, context 32768, bf16 cache",
     "v2_b2_l128k_fp8": "V2 dims, batch 2, context 131072, e4m3 cache with per-token fp32 scale",
 }
-STAGES = ("append", "absorb", "decode_partial", "decode_combine", "out_proj")
+STAGES = ("append", "absorb", "decode_partial", "combine_out_proj")   # DecodeStep.stages()
 # the sources that define each tensor-core stage's kernel (its device code, the
 # PTX wrappers it uses and its launcher): a traffic figure taken by ncu is only
 # reported while all of them are unchanged
@@ -50,6 +51,9 @@ KERNEL_FILES = {
     "decode_partial": ["mla_latent_kv_19_b200/csrc/decode_umma.cuh",
                        "mla_latent_kv_19_b200/csrc/sm100_ptx.cuh",
                        "mla_latent_kv_19_b200/csrc/umma_kernels.cu"],
+    "combine_out_proj": ["mla_latent_kv_19_b200/csrc/gemm_umma.cuh",
+                         "mla_latent_kv_19_b200/csrc/sm100_ptx.cuh",
+                         "mla_latent_kv_19_b200/csrc/umma_kernels.cu"],
     "out_proj": ["mla_latent_kv_19_b200/csrc/gemm_umma.cuh",
                  "mla_latent_kv_19_b200/csrc/sm100_ptx.cuh",
                  "mla_latent_kv_19_b200/csrc/umma_kernels.cu"],
@@ -82,9 +86,10 @@ def algorithmic(wl, S):
                        flops=2 * B * H * dn * dc),
         "decode_partial": dict(bytes=tokens * row + B * H * D * a + B * H * dc * a,
                                flops=2 * H * (D + dc) * tokens),
-        "decode_combine": dict(bytes=B * S * H * (dc + 1) * 4 + B * H * dc * a + B * H * 4, flops=0),
-        "out_proj": dict(bytes=H * dv * dc * a + dm * H * dv * a + B * H * dc * a + B * dm * a,
-                         flops=2 * B * H * dv * dc + 2 * B * dm * H * dv),
+        # merge + output projection: the weights, o_lat and lse written, y written
+        # (the split partials it reads are the decode's scratch, not counted)
+        "combine_out_proj": dict(bytes=H * dv * dc * a + dm * H * dv * a + B * H * dc * a + B * H * 4 + B * dm * a,
+                                 flops=2 * B * H * dv * dc + 2 * B * dm * H * dv),
     }
     return out, tokens
 
@@ -269,7 +274,7 @@ def main():
     timed = torch.cuda.CUDAGraph()
     with torch.cuda.graph(timed):
         ev[0].record()
-        for i, fn in enumerate((st.append, st.absorb, st.decode_partial, st.decode_combine, st.out_proj)):
+        for i, (_, fn) in enumerate(st.stages()):
             fn()
             ev[i + 1].record()
     torch.cuda.synchronize(dev)
@@ -332,7 +337,7 @@ def main():
 
     alg, tokens = algorithmic(wl, st.num_splits)
     hbm, bf16, bf16_sus, peak_kind = measured_peaks()
-    dom = max(("decode_partial", "out_proj", "absorb"), key=lambda s: stage_ms[s])
+    dom = max(("decode_partial", "combine_out_proj", "absorb"), key=lambda s: stage_ms[s])
     kernels = {}
     for s in STAGES:
         t = stage_ms[s] / 1e3
@@ -365,7 +370,7 @@ def main():
         "kernels": kernels,
         "roofline": roof,
         "gpu_launches": int(launches),
-        "graphs": "each timed step is one replay of a CUDA graph of the five C-ABI calls, with timing "
+        "graphs": "each timed step is one replay of a CUDA graph of the step's C-ABI calls, with timing "
                   "events recorded inside it between the stages; e2e replays the same step graph",
         "clocks": clk,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),

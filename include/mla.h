@@ -241,6 +241,23 @@ MLA_API int mla_out_proj(mla_handle_t h, const void* o_lat, const void* w_uv, co
                  int32_t batch, void* workspace, size_t workspace_bytes, void* y, void* o_out,
                  cudaStream_t stream);
 
+/* mla_combine_out_proj -- the split merge of mla_decode_combine followed by
+ * mla_out_proj, in one call (V2 page section 2.3 for the output side; the merge
+ * is the log-sum-exp combination of the split partials).  Where the tensor-core
+ * path covers the batch, the merge runs inside the W_UV kernel: every head's
+ * merged o_lat slice is built straight into that kernel's operand, which saves
+ * the merge kernel and its round trip through memory; the results are bit-for-
+ * bit those of the two separate calls.  Otherwise the two calls run in turn.
+ * batch / max_seq_len / num_splits / workspace as for mla_decode_partial (its
+ * workspace holds the partials); w_uv, w_o, op_workspace (at least
+ * mla_out_proj_workspace_bytes), y and o_out as for mla_out_proj; o_lat
+ * [batch, H, d_c] out (required); lse [batch, H] out or NULL.
+ * Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, LAUNCH. */
+MLA_API int mla_combine_out_proj(mla_handle_t h, int32_t batch, int32_t max_seq_len, int32_t num_splits,
+                                 const void* workspace, size_t workspace_bytes, const void* w_uv,
+                                 const void* w_o, void* op_workspace, size_t op_workspace_bytes,
+                                 void* o_lat, float* lse, void* y, void* o_out, cudaStream_t stream);
+
 /* Synchronise the stream, then read and clear the handle's device error word:
  * MLA_OK, MLA_ERR_BAD_INDEX or MLA_ERR_TIMEOUT (or MLA_ERR_CUDA if the sync
  * itself failed).  Not for use inside stream capture. */

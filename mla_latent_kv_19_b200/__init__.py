@@ -67,6 +67,7 @@ _SIGS = {
     "mla_decode_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _P, _P, _P]),
     "mla_out_proj_workspace_bytes": (_SZ, [_P, _I]),
     "mla_out_proj": (ctypes.c_int, [_P, _P, _P, _P, _I, _P, _SZ, _P, _P, _P]),
+    "mla_combine_out_proj": (ctypes.c_int, [_P, _I, _I, _I, _P, _SZ, _P, _P, _P, _SZ, _P, _P, _P, _P, _P]),
     "mla_last_device_error": (ctypes.c_int, [_P, _P]),
     "mla_set_wait_limit": (ctypes.c_int, [_P, ctypes.c_uint32]),
     "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -245,6 +246,14 @@ def mla_out_proj(h: Handle, o_lat, w_uv, w_o, workspace, y, o_out=None, stream=N
     _check("mla_out_proj", lib.mla_out_proj(
         h.ptr, _ptr(o_lat), _ptr(w_uv), _ptr(w_o), o_lat.shape[0], _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(y), _ptr(o_out), _stream(stream)))
+
+
+def mla_combine_out_proj(h: Handle, batch: int, max_seq_len: int, num_splits: int, workspace, w_uv, w_o,
+                         op_workspace, o_lat, y, lse=None, o_out=None, stream=None) -> None:
+    _check("mla_combine_out_proj", lib.mla_combine_out_proj(
+        h.ptr, batch, max_seq_len, num_splits, _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(w_uv), _ptr(w_o), _ptr(op_workspace), op_workspace.numel() * op_workspace.element_size(),
+        _ptr(o_lat), _ptr(lse), _ptr(y), _ptr(o_out), _stream(stream)))
 
 
 def mla_last_device_error(h: Handle, stream=None) -> int:

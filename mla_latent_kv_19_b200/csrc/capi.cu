@@ -397,6 +397,47 @@ int mla_out_proj(mla_handle_t h, const void* o_lat, const void* w_uv, const void
   return map_cuda(launch_out_proj_generic(a, h->cfg.act_dtype, stream));
 }
 
+int mla_combine_out_proj(mla_handle_t h, int32_t batch, int32_t max_seq_len, int32_t num_splits,
+                         const void* workspace, size_t workspace_bytes, const void* w_uv,
+                         const void* w_o, void* op_workspace, size_t op_workspace_bytes,
+                         void* o_lat, float* lse, void* y, void* o_out, cudaStream_t stream) {
+  int S = 0;
+  int st = decode_check(h, batch, max_seq_len, num_splits, workspace, workspace_bytes, &S);
+  if (st != MLA_OK || batch == 0) return st;
+  if (o_lat == nullptr || w_uv == nullptr || w_o == nullptr || y == nullptr) return MLA_ERR_INVALID_ARG;
+  if (op_workspace == nullptr || op_workspace_bytes < mla_out_proj_workspace_bytes(h, batch))
+    return MLA_ERR_WORKSPACE;
+  if (!aligned(o_lat, 16) || (lse && !aligned(lse, 4)) || !aligned(w_uv, 16) || !aligned(w_o, 16) ||
+      !aligned(y, 16) || !aligned(op_workspace, 16) || (o_out && !aligned(o_out, 16)))
+    return MLA_ERR_ALIGNMENT;
+  if (!umma_combine_out_proj_supported(h, batch, S)) {
+    // the merge and the output projection as two calls
+    st = mla_decode_combine(h, batch, max_seq_len, num_splits, workspace, workspace_bytes, o_lat, lse, stream);
+    if (st != MLA_OK) return st;
+    return mla_out_proj(h, o_lat, w_uv, w_o, batch, op_workspace, op_workspace_bytes, y, o_out, stream);
+  }
+  const size_t parts = static_cast<size_t>(batch) * S * h->cfg.num_heads;
+  OutProjArgs a{};
+  a.o_lat = o_lat;
+  a.w_uv = w_uv;
+  a.w_o = w_o;
+  a.o = o_out ? o_out : op_workspace;
+  a.y = y;
+  a.batch = batch;
+  a.num_heads = h->cfg.num_heads;
+  a.d_c = h->cfg.d_c;
+  a.d_v = h->cfg.d_v;
+  a.d_model = h->cfg.d_model;
+  a.comb_opart = static_cast<const float*>(workspace);
+  a.comb_lse = reinterpret_cast<const float*>(static_cast<const char*>(workspace) +
+                                              round_up(parts * h->cfg.d_c * sizeof(float), 256));
+  a.comb_splits = S;
+  a.comb_lse_out = lse;
+  void* extra = static_cast<char*>(op_workspace) +
+                round_up(static_cast<size_t>(batch) * h->cfg.num_heads * h->cfg.d_v * act_bytes(h->cfg.act_dtype), 256);
+  return map_cuda(launch_out_proj_umma(h, a, extra, stream));
+}
+
 int mla_last_device_error(mla_handle_t h, cudaStream_t stream) {
   if (h == nullptr) return MLA_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return MLA_ERR_CUDA;

@@ -60,9 +60,20 @@ struct Params {
   const int32_t* pos;
   const float2* rope_cs;
   int num_heads, d_c, d_r, max_position;
+  // W_UV fed straight from split-KV partials: the resident X slice o_lat[:, h, :]
+  // is merged in the kernel (log-sum-exp weights, as the merge kernel computes
+  // them) instead of being loaded; comb_splits = 0 turns this off
+  const float* comb_opart;     // o_part [batch][S][d_c/4][H][4]
+  const float* comb_lse;       // lse_part [batch][S][H]
+  int comb_splits;             // S
+  __nv_bfloat16* comb_olat;    // optional: o_lat [batch][H][d_c] is written too
+  float* comb_lse_out;         // optional: lse [batch][H]
   int* err;
   uint32_t wait_limit;
 };
+
+// Threads of the CTA that build a merged X slice (warps 2..7).
+constexpr int kCombThreads = 192;
 
 template <bool kAMn, Epi kEpi>
 __global__ void __launch_bounds__(256, 1)
@@ -95,8 +106,11 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t done = bars + 8u * (2 * p.stages);
   const uint32_t drainb = done + 8u;
   const uint32_t xfull = drainb + 8u;
+  const uint32_t wready = xfull + 8u;
+  const bool xcomb = xres && p.comb_splits > 0;
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + xres_bytes + p.stages * stage_bytes +
-                                                                 8 * (2 * p.stages + 3));
+                                                                 8 * (2 * p.stages + 4));
+  float* wts = reinterpret_cast<float*>(smem + xres_bytes + p.stages * stage_bytes + 8 * (2 * p.stages + 4) + 16);
   // TMEM: one block of ncpt columns per M tile
   const uint32_t ncpt = p.n <= 32 ? 32u : (p.n <= 64 ? 64u : (p.n <= 128 ? 128u : 256u));
   uint32_t ncols = 32;
@@ -108,7 +122,8 @@ __global__ void __launch_bounds__(256, 1)
     }
     ptx::mbar_init(done, 1);
     ptx::mbar_init(drainb, 1);
-    ptx::mbar_init(xfull, 1);
+    ptx::mbar_init(xfull, xcomb ? kCombThreads : 1);
+    ptx::mbar_init(wready, kCombThreads);
     misc[1] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -137,7 +152,7 @@ __global__ void __launch_bounds__(256, 1)
     if (lane == 0) {
       ptx::prefetch_tmap(&tmA);
       ptx::prefetch_tmap(&tmX);
-      if (xres && nst > 0) {
+      if (xres && !xcomb && nst > 0) {
         // the CTA's whole slice of X, once
         ptx::mbar_arrive_expect_tx(xfull, xres_bytes);
         ptx::tma_load_3d(sb, &tmX, xfull, 0, 0, (group * p.x_col_group) / kKc + kc0);
@@ -161,7 +176,7 @@ __global__ void __launch_bounds__(256, 1)
       }
       for (int i = max(0, issued - p.stages); i < issued; ++i)
         ptx::mbar_wait<false>(full(i % p.stages), (i / p.stages) & 1, 0xffffffffu, kWaitNs);
-      if (xres && nst > 0) ptx::mbar_wait<false>(xfull, 0, 0xffffffffu, kWaitNs);
+      if (xres && !xcomb && nst > 0) ptx::mbar_wait<false>(xfull, 0, 0xffffffffu, kWaitNs);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -195,7 +210,66 @@ __global__ void __launch_bounds__(256, 1)
       ptx::mbar_wait<false>(drainb, 0, 0xffffffffu, kWaitNs);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  }
+  if (xcomb && warp >= 2) {
+    // merge this group's (head's) split partials into the resident X slice:
+    // o_lat[b][c] = sum_s exp(lse_s - m) o_part_s[b][c] / sum_s exp(lse_s - m),
+    // with m = max_s lse_s, in the same order and precision as the merge kernel
+    const int ct = static_cast<int>(threadIdx.x) - 64;
+    const int S = p.comb_splits, H = p.num_heads, h = group;
+    float* invz = wts + p.n * S;
+    for (int b = ct; b < p.n; b += kCombThreads) {
+      float mm = -INFINITY;
+      if (b < p.batch)
+        for (int sp = 0; sp < S; ++sp) mm = fmaxf(mm, p.comb_lse[(static_cast<long>(b) * S + sp) * H + h]);
+      float z = 0.f;
+      for (int sp = 0; sp < S; ++sp) {
+        const float w = (b >= p.batch || mm == -INFINITY) ? 0.f
+                                                           : __expf(p.comb_lse[(static_cast<long>(b) * S + sp) * H + h] - mm);
+        wts[b * S + sp] = w;
+        z += w;
+      }
+      invz[b] = z > 0.f ? 1.f / z : 0.f;
+      if (p.comb_lse_out != nullptr && b < p.batch)
+        p.comb_lse_out[static_cast<long>(b) * H + h] = z > 0.f ? mm + __logf(z) : -INFINITY;
+    }
+    ptx::mbar_arrive(wready);
+    const bool wok = wait(wready, 0);
+    if (wok) {
+      const int dq = p.d_c / 4;
+      const float4* op = reinterpret_cast<const float4*>(p.comb_opart);
+      for (int u = ct; u < p.n * 8 * p.x_chunks; u += kCombThreads) {
+        // 16-byte unit u: row b, K chunk k, unit v (columns 64k + 8v .. +7)
+        const int b = u / (8 * p.x_chunks), k = (u / 8) % p.x_chunks, v = u % 8;
+        const int g0 = (64 * k + 8 * v) / 4;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        if (b < p.batch) {
+          for (int sp = 0; sp < S; ++sp) {
+            const float w = wts[b * S + sp];
+            const float4* os = op + ((static_cast<long>(b) * S + sp) * dq + g0) * H + h;
+            const float4 x0 = os[0], x1 = os[H];
+            acc[0] += w * x0.x; acc[1] += w * x0.y; acc[2] += w * x0.z; acc[3] += w * x0.w;
+            acc[4] += w * x1.x; acc[5] += w * x1.y; acc[6] += w * x1.z; acc[7] += w * x1.w;
+          }
+        }
+        uint4 pk;
+        uint32_t* pw = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 bb = __floats2bfloat162_rn(acc[2 * e] * invz[b], acc[2 * e + 1] * invz[b]);
+          pw[e] = *reinterpret_cast<const uint32_t*>(&bb);
+        }
+        *reinterpret_cast<uint4*>(smem + k * (p.n * 128) + b * 128 + ((v ^ (b & 7)) << 4)) = pk;
+        if (p.comb_olat != nullptr && b < p.batch)
+          *reinterpret_cast<uint4*>(p.comb_olat + (static_cast<long>(b) * H + h) * p.d_c + 64 * k + 8 * v) = pk;
+      }
+    }
+    ptx::fence_proxy_async_cta();     // generic writes -> the MMAs' reads of X
+    ptx::mbar_arrive(xfull);
+  }
+  if (warp >= 4) {
     const int q = warp & 3;
     const int m = q * 32 + lane;                       // row of this thread in a tile
     const uint32_t lb = static_cast<uint32_t>(q * 32) << 16;

@@ -87,6 +87,12 @@ struct OutProjArgs {
   void* o;             // [B, H, d_v]
   void* y;             // [B, d_model]
   int32_t batch, num_heads, d_c, d_v, d_model;
+  // merge fused into W_UV: o_lat (then an output) is built from the split-KV
+  // partials; comb_splits = 0 turns this off
+  const float* comb_opart;   // [B, S, d_c/4, H, 4]
+  const float* comb_lse;     // [B, S, H]
+  int32_t comb_splits;
+  float* comb_lse_out;       // [B, H] or null
 };
 
 // Launchers (return cudaGetLastError() of their launches).

@@ -120,7 +120,9 @@ int padded_n(int batch) { return (batch + 15) / 16 * 16; }
 size_t gemm_smem_bytes(const gemm::Params& p) {
   const size_t xres = p.x_chunks > 0 ? static_cast<size_t>(p.n) * gemm::kKc * 2 * p.x_chunks : 0;
   const size_t stage = gemm::kM * gemm::kKc * 2 * p.kcs + (p.x_chunks > 0 ? 0 : p.n * gemm::kKc * 2 * p.kcs);
-  return xres + static_cast<size_t>(p.stages) * stage + 8 * (2 * p.stages + 3) + 16 + 1024;
+  // merge weights [n][S] and 1/z [n] when the merge runs in the kernel
+  const size_t wts = p.comb_splits > 0 ? static_cast<size_t>(p.n) * (p.comb_splits + 1) * 4 : 0;
+  return xres + static_cast<size_t>(p.stages) * stage + 8 * (2 * p.stages + 4) + 16 + wts + 1024;
 }
 
 // Raise a kernel's dynamic shared-memory limit once (per process) to the
@@ -223,6 +225,15 @@ bool umma_out_proj_supported(const mla_ctx* h, int batch) {
   return v2_bf16(h) && batch >= 1 && batch <= 256;
 }
 
+bool umma_combine_out_proj_supported(const mla_ctx* h, int batch, int num_splits) {
+  if (!umma_out_proj_supported(h, batch) || num_splits < 1 || h->cfg.num_heads > 128) return false;
+  // the W_UV kernel keeps the merged slice resident: X, two 64 KB weight boxes
+  // and the merge weights must fit in shared memory
+  const long n = padded_n(batch);
+  const long bytes = n * h->cfg.d_c * 2 + 2L * gemm::kM * gemm::kKc * 2 * 4 + n * (num_splits + 1) * 4 + 4096;
+  return bytes <= 232448;
+}
+
 size_t umma_out_proj_extra_workspace(const mla_ctx* h, int batch) {
   if (!umma_out_proj_supported(h, batch)) return 0;
   return static_cast<size_t>(kOProjSplits) * batch * h->cfg.d_model * sizeof(float) + 256;
@@ -233,9 +244,12 @@ cudaError_t launch_out_proj_umma(const mla_ctx* h, const OutProjArgs& a, void* e
   const int H = a.num_heads, n = padded_n(a.batch);
   const long kdim = static_cast<long>(H) * a.d_v;
   // o[b][h][v] = W_UV[h] o_lat[b][h]: one CTA per head; while the head's o_lat
-  // slice fits next to two 64 KB weight boxes it is loaded once and kept
+  // slice fits next to two 64 KB weight boxes it is loaded once and kept -- or,
+  // with the merge fused, built in the kernel from the split partials
   {
     const bool xres = static_cast<long>(n) * a.d_c * 2 + 2L * gemm::kM * gemm::kKc * 2 * 4 + 4096 <= 232448;
+    if (a.comb_splits > 0 && !umma_combine_out_proj_supported(h, a.batch, a.comb_splits))
+      return cudaErrorNotSupported;
     const int kcs = xres ? 4 : 2;
     CUtensorMap ta, tx;
     cudaError_t e = make_map_rows_chunked(&ta, a.w_uv, static_cast<uint64_t>(H) * a.d_v, a.d_c * 2,
@@ -259,6 +273,15 @@ cudaError_t launch_out_proj_umma(const mla_ctx* h, const OutProjArgs& a, void* e
     p.out = a.o;
     p.out_ld = kdim;
     p.out_group = a.d_v;
+    p.num_heads = H;
+    p.d_c = a.d_c;
+    if (a.comb_splits > 0) {
+      p.comb_opart = a.comb_opart;
+      p.comb_lse = a.comb_lse;
+      p.comb_splits = a.comb_splits;
+      p.comb_olat = static_cast<__nv_bfloat16*>(const_cast<void*>(a.o_lat));
+      p.comb_lse_out = a.comb_lse_out;
+    }
     p.err = h->err;
     p.wait_limit = h->wait_limit;
     e = launch_gemm<false, gemm::Epi::kStoreBf16T>(ta, tx, p, dim3(H, 1), s);

@@ -16,7 +16,7 @@ from typing import Dict, Optional
 import numpy as np
 import torch
 
-from . import (Handle, mla_absorb_q, mla_cache_append, mla_decode_auto_splits,
+from . import (Handle, mla_absorb_q, mla_cache_append, mla_combine_out_proj, mla_decode_auto_splits,
                mla_decode_combine, mla_decode_partial, mla_decode_workspace_bytes,
                mla_kv_project_append, mla_out_proj, mla_out_proj_workspace_bytes)
 
@@ -153,12 +153,21 @@ class DecodeStep:
         mla_out_proj(self.h, self.o_lat, self.w_uv, self.w_o, self.op_ws, self.y, self.o,
                      stream=stream)
 
+    def combine_out_proj(self, stream=None) -> None:
+        """The split merge and the output projection in one call (the merge runs
+        inside the W_UV kernel where the library can)."""
+        mla_combine_out_proj(self.h, self.B, self.max_seq_len, self.num_splits, self.dec_ws, self.w_uv,
+                             self.w_o, self.op_ws, self.o_lat, self.y, lse=self.lse, o_out=self.o,
+                             stream=stream)
+
+    def stages(self):
+        """(name, call) of the C-ABI calls of one decode step, in order."""
+        return [("append", self.append), ("absorb", self.absorb), ("decode_partial", self.decode_partial),
+                ("combine_out_proj", self.combine_out_proj)]
+
     def run(self, stream=None) -> None:
-        self.append(stream)
-        self.absorb(stream)
-        self.decode_partial(stream)
-        self.decode_combine(stream)
-        self.out_proj(stream)
+        for _, fn in self.stages():
+            fn(stream)
 
     # -- CUDA graphs of the step (the C-ABI calls neither allocate nor sync) --
     def capture(self) -> None:
@@ -167,7 +176,7 @@ class DecodeStep:
         buffers of this object: refresh inputs in place (copy_) between replays."""
         torch.cuda.synchronize(self.device)
         self.stage_graphs = []
-        for fn in (self.append, self.absorb, self.decode_partial, self.decode_combine, self.out_proj):
+        for _, fn in self.stages():
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
                 fn()

@@ -69,3 +69,39 @@ def test_out_proj_against_oracle(batch):
     r_y = oracle.out_project(r_o, wl.to_f64(wl.w_o))
     assert_close("o", g_o, r_o)
     assert_close("y", g_y, r_y)
+
+
+@pytest.mark.parametrize("name,kw,splits", [
+    ("v2_b32_l2048", dict(batch=5, context=700), 3),
+    ("v2_b32_l2048", dict(batch=32, context=300), 2),
+    ("v2_b2_l128k_fp8", dict(batch=2, context=3000), 8),
+    ("v2_b32_l2048", dict(batch=100, context=64), 1),      # beyond the fused path: two calls
+])
+def test_fused_merge_out_proj_equals_the_two_calls(name, kw, splits):
+    """mla_combine_out_proj (the split merge built inside the W_UV kernel) gives
+    bit for bit what mla_decode_combine followed by mla_out_proj gives, and
+    both match the oracle."""
+    from mla_latent_kv_19_b200 import mla_combine_out_proj, mla_last_device_error
+    from mla_latent_kv_19_b200.step import DecodeStep
+    wl = workloads.make(name, **kw)
+    st = DecodeStep(wl, num_splits=splits)
+    st.append()
+    st.absorb()
+    st.decode_partial()
+    st.decode_combine()
+    st.out_proj()
+    sep = {k: getattr(st, k).clone() for k in ("o_lat", "lse", "o", "y")}
+    out = {k: torch.full_like(v, float("nan")) for k, v in sep.items()}
+    mla_combine_out_proj(st.h, st.B, st.max_seq_len, st.num_splits, st.dec_ws, st.w_uv, st.w_o, st.op_ws,
+                         out["o_lat"], out["y"], lse=out["lse"], o_out=out["o"])
+    assert mla_last_device_error(st.h) == 0
+    torch.cuda.synchronize()
+    for k in sep:
+        assert torch.equal(out[k].view(torch.int16) if out[k].dtype == torch.bfloat16 else out[k],
+                           sep[k].view(torch.int16) if sep[k].dtype == torch.bfloat16 else sep[k]), k
+    st.close()
+    fp8 = wl.cache_dtype == "fp8_e4m3"
+    r = oracle.step_outputs(wl, fp8_dequant=fp8)
+    g = {k: v.float().cpu().numpy() for k, v in out.items()}
+    for k in ("o_lat", "lse", "y"):
+        assert_close(k, g[k], r[k])
