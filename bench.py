@@ -229,6 +229,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--overlap", action="store_true",
+                    help="launch each kernel as a programmatic dependent of the one before it")
     ap.add_argument("--ref-seconds", type=float, default=10.0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -249,7 +251,7 @@ def main():
     base_seed = {"v2_b32_l2048": 1, "v2_ragged64": 2, "v2_b4_l32k": 3, "v2_b2_l128k_fp8": 4}.get(args.workload, 1)
     wl = workloads.make(args.workload, seed=dist.rank_seed(base_seed, rank))
     dev = torch.device("cuda", local)
-    st = DecodeStep(wl, device=dev, num_splits=args.num_splits)
+    st = DecodeStep(wl, device=dev, num_splits=args.num_splits, overlap=args.overlap)
     stream = torch.cuda.current_stream(dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
@@ -263,25 +265,36 @@ def main():
         torch.sum(flush, dim=0, dtype=torch.int64, out=flush_sum)
 
     # one eager step configures the kernels and counts this library's launches per
-    # step; the timed steps replay ONE CUDA graph of the whole step, with timing
-    # events recorded inside it between the stages (graph event-record nodes)
+    # step.  Each timed step replays ONE CUDA graph of the whole step with timing
+    # events at its two ends only (an event between two kernels would end the
+    # overlap of the second's launch with the first); the per-stage breakdown
+    # comes from a second graph of the same step with events between the stages,
+    # replayed after it (with its own L2 flush)
     l0 = mla_launch_count()
     st.run(stream)
     torch.cuda.synchronize(dev)
     launches_per_step = mla_launch_count() - l0
     st.capture()
-    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(STAGES) + 1)]
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
     timed = torch.cuda.CUDAGraph()
     with torch.cuda.graph(timed):
         ev[0].record()
+        st.run()
+        ev[1].record()
+    sev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(STAGES) + 1)]
+    staged = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(staged):
+        sev[0].record()
         for i, (_, fn) in enumerate(st.stages()):
             fn()
-            ev[i + 1].record()
+            sev[i + 1].record()
     torch.cuda.synchronize(dev)
 
     for _ in range(args.warmup):
         flush_l2()
         timed.replay()
+        flush_l2()
+        staged.replay()
     torch.cuda.synchronize(dev)
 
     clocks = ClockSampler(local)
@@ -294,8 +307,11 @@ def main():
         flush_l2()                         # L2 flush, outside the step's events
         timed.replay()
         torch.cuda.synchronize(dev)        # read this replay's events before the next one
-        step_ms.append(ev[0].elapsed_time(ev[-1]))
-        stage_rows.append([ev[i].elapsed_time(ev[i + 1]) for i in range(len(STAGES))])
+        step_ms.append(ev[0].elapsed_time(ev[1]))
+        flush_l2()
+        staged.replay()
+        torch.cuda.synchronize(dev)
+        stage_rows.append([sev[i].elapsed_time(sev[i + 1]) for i in range(len(STAGES))])
     torch.cuda.synchronize(dev)
     dist.barrier()
     launches = launches_per_step * args.steps
@@ -361,6 +377,7 @@ def main():
         "config": {"workload": f"{args.workload}: {WORKLOAD_TEXT.get(args.workload, '')}",
                    "batch_per_gpu": wl.batch, "tokens_per_gpu": tokens, "num_splits": st.num_splits,
                    "parallelism": f"data parallel over sequences, {world} rank(s), no collective on the path",
+                   "launch_overlap": args.overlap,
                    "l2": "flushed before every step (write of 2x L2 size, then a read of it so that no dirty "
                          "line is left to write back), outside the step's events"},
         "decode": {"us": t_dec * 1e6, "latent_cache_GB/s": dec["bytes"] / t_dec / 1e9,
@@ -370,8 +387,10 @@ def main():
         "kernels": kernels,
         "roofline": roof,
         "gpu_launches": int(launches),
-        "graphs": "each timed step is one replay of a CUDA graph of the step's C-ABI calls, with timing "
-                  "events recorded inside it between the stages; e2e replays the same step graph",
+        "graphs": "each timed step is one replay of a CUDA graph of the step's C-ABI calls (kernels "
+                  "launched as programmatic dependents of the one before), timed by events at its two "
+                  "ends; the per-stage times come from a second graph with events between the stages, "
+                  "replayed after it; e2e replays the step graph",
         "clocks": clk,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_s * 1e3},

@@ -227,6 +227,23 @@ MLA_API int mla_decode_noalloc(mla_handle_t h, const void* q_lat, const void* ca
                                const int32_t* seq_lens, int32_t batch, int32_t max_seq_len,
                                int32_t num_splits, void* o_lat, float* lse, cudaStream_t stream);
 
+/* W_O in tile-major order, for a faster weight stream.  Writes
+ * w_o_tiled[m/128][k/64][m%128][k%64] = w_o[m][k] for the handle's
+ * [d_model, H*d_v] W_O (act dtype), so that every 128 x 64 tile is one
+ * contiguous 16 KB (32 KB in fp32) run; the tensor-core output projection then
+ * reads one contiguous run per request.  w_o_tiled is a separate buffer of the
+ * same size, owned by the caller; both 16-byte aligned.  Asynchronous on
+ * `stream`.  Errors: INVALID_ARG (null or identical pointers), UNSUPPORTED
+ * (d_model not a multiple of 128 or H*d_v not a multiple of 64), ALIGNMENT,
+ * LAUNCH. */
+MLA_API int mla_pack_w_o(mla_handle_t h, const void* w_o, void* w_o_tiled, cudaStream_t stream);
+
+/* Layout of the w_o argument of later mla_out_proj / mla_combine_out_proj
+ * calls on this handle: 0 row-major (default), 1 tile-major (mla_pack_w_o).
+ * Results do not depend on the layout beyond fp32 summation order.  Errors:
+ * INVALID_ARG (null handle), UNSUPPORTED (shape not tileable). */
+MLA_API int mla_set_w_o_layout(mla_handle_t h, int tiled);
+
 /* Workspace bytes mla_out_proj needs for this batch. */
 MLA_API size_t mla_out_proj_workspace_bytes(mla_handle_t h, int32_t batch);
 
@@ -234,7 +251,8 @@ MLA_API size_t mla_out_proj_workspace_bytes(mla_handle_t h, int32_t batch);
  * two contractions:  o[b][h] = W_UV[h] o_lat[b][h]  (d_v x d_c per head), then
  * y[b] = W_O concat_h o[b][h]  (d_model x H*d_v).  fp32 accumulation; o is
  * rounded to the act dtype between the two.
- * o_lat [batch, H, d_c]; w_uv [H, d_v, d_c]; w_o [d_model, H*d_v];
+ * o_lat [batch, H, d_c]; w_uv [H, d_v, d_c]; w_o [d_model, H*d_v] row-major,
+ * or tile-major after mla_set_w_o_layout(h, 1) (see mla_pack_w_o);
  * y [batch, d_model] out; o_out [batch, H, d_v] out, or NULL to keep o in the
  * workspace only.  Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, LAUNCH. */
 MLA_API int mla_out_proj(mla_handle_t h, const void* o_lat, const void* w_uv, const void* w_o,
@@ -267,6 +285,18 @@ MLA_API int mla_last_device_error(mla_handle_t h, cudaStream_t stream);
  * device-side wait loop (0 = the built-in default).  A limit so small that a
  * wait gives up makes the kernel record MLA_ERR_TIMEOUT and return. */
 MLA_API int mla_set_wait_limit(mla_handle_t h, uint32_t limit);
+
+/* Launch overlap (programmatic dependent launch), off by default.  When on,
+ * each kernel of this handle is launched so that it may start while the
+ * kernel issued before it on the same stream is still running: it sets up its
+ * barriers and tensor memory and requests its first weight boxes (W_UK for
+ * mla_absorb_q, W_UV and W_O for mla_out_proj / mla_combine_out_proj), then
+ * waits for that kernel to complete before it reads any other input or writes
+ * any output.  The caller's obligation: the weight operands of a call must not
+ * be written by the kernel issued immediately before it on the stream.  Every
+ * other input may come from that kernel.  Returns MLA_OK or
+ * MLA_ERR_INVALID_ARG (null handle). */
+MLA_API int mla_set_launch_overlap(mla_handle_t h, int enable);
 
 /* Number of kernels this library has launched in this process (all handles,
  * all devices), for accounting of launches over a timed region. */

@@ -21,7 +21,8 @@ __all__ = [
     "mla_decode", "mla_decode_partial", "mla_decode_combine", "mla_decode_auto_splits",
     "mla_decode_noalloc",
     "mla_decode_workspace_bytes", "mla_out_proj", "mla_out_proj_workspace_bytes",
-    "mla_last_device_error", "mla_set_wait_limit", "mla_status_string", "mla_launch_count",
+    "mla_last_device_error", "mla_set_wait_limit", "mla_set_launch_overlap", "mla_status_string",
+    "mla_launch_count", "mla_combine_out_proj", "mla_pack_w_o", "mla_set_w_o_layout",
     "MLA_BF16", "MLA_FP8_E4M3", "MLA_FP32", "EXPORTED_SYMBOLS",
 ]
 
@@ -70,6 +71,9 @@ _SIGS = {
     "mla_combine_out_proj": (ctypes.c_int, [_P, _I, _I, _I, _P, _SZ, _P, _P, _P, _SZ, _P, _P, _P, _P, _P]),
     "mla_last_device_error": (ctypes.c_int, [_P, _P]),
     "mla_set_wait_limit": (ctypes.c_int, [_P, ctypes.c_uint32]),
+    "mla_set_launch_overlap": (ctypes.c_int, [_P, ctypes.c_int]),
+    "mla_pack_w_o": (ctypes.c_int, [_P, _P, _P, _P]),
+    "mla_set_w_o_layout": (ctypes.c_int, [_P, ctypes.c_int]),
     "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_launch_count": (ctypes.c_uint64, []),
 }
@@ -266,3 +270,19 @@ def mla_launch_count() -> int:
 
 def mla_set_wait_limit(h: Handle, limit: int) -> None:
     _check("mla_set_wait_limit", lib.mla_set_wait_limit(h.ptr, limit))
+
+
+def mla_pack_w_o(h: Handle, w_o, w_o_tiled, stream=None) -> None:
+    """w_o_tiled <- W_O in tile-major order ([d_model/128][H*d_v/64][128][64])."""
+    _check("mla_pack_w_o", lib.mla_pack_w_o(h.ptr, _ptr(w_o), _ptr(w_o_tiled), _stream(stream)))
+
+
+def mla_set_w_o_layout(h: Handle, tiled: bool) -> None:
+    """Whether later output projections on h read a tile-major w_o."""
+    _check("mla_set_w_o_layout", lib.mla_set_w_o_layout(h.ptr, 1 if tiled else 0))
+
+
+def mla_set_launch_overlap(h: Handle, enable: bool) -> None:
+    """Launch this handle's kernels as programmatic dependents of the kernel
+    before them on the stream (weights are then read before that kernel ends)."""
+    _check("mla_set_launch_overlap", lib.mla_set_launch_overlap(h.ptr, 1 if enable else 0))

@@ -115,6 +115,8 @@ int mla_create(const mla_config_t* cfg, mla_handle_t* out) {
   h->cc_major = prop.major;
   h->cc_minor = prop.minor;
   h->wait_limit = kDefaultWaitLimit;
+  h->overlap = 0;
+  h->w_o_tiled = 0;
   if (cudaMalloc(&h->rope_cs, table.size() * sizeof(float2)) != cudaSuccess ||
       cudaMalloc(&h->err, 256) != cudaSuccess ||
       cudaMemcpy(h->rope_cs, table.data(), table.size() * sizeof(float2),
@@ -197,6 +199,7 @@ static int append_common(mla_handle_t h, const void* c_kv, const void* k_r, cons
   a.d_model = h->cfg.d_model;
   a.block_size = h->cfg.block_size;
   a.max_position = h->cfg.max_position;
+  a.overlap = h->overlap;
   return map_cuda(launch_append(a, h->cfg.act_dtype, h->cfg.cache_dtype, project, stream));
 }
 
@@ -338,6 +341,7 @@ int mla_decode_combine(mla_handle_t h, int32_t batch, int32_t max_seq_len, int32
   a.num_heads = h->cfg.num_heads;
   a.d_c = h->cfg.d_c;
   a.num_splits = S;
+  a.overlap = h->overlap;
   return map_cuda(launch_combine(a, h->cfg.act_dtype, h->num_sms, stream));
 }
 
@@ -387,6 +391,7 @@ int mla_out_proj(mla_handle_t h, const void* o_lat, const void* w_uv, const void
   a.d_c = h->cfg.d_c;
   a.d_v = h->cfg.d_v;
   a.d_model = h->cfg.d_model;
+  a.w_o_tiled = h->w_o_tiled;
   if (umma_out_proj_supported(h, batch)) {
     void* extra = static_cast<char*>(workspace) +
                   round_up(static_cast<size_t>(batch) * h->cfg.num_heads * h->cfg.d_v *
@@ -433,6 +438,7 @@ int mla_combine_out_proj(mla_handle_t h, int32_t batch, int32_t max_seq_len, int
                                               round_up(parts * h->cfg.d_c * sizeof(float), 256));
   a.comb_splits = S;
   a.comb_lse_out = lse;
+  a.w_o_tiled = h->w_o_tiled;
   void* extra = static_cast<char*>(op_workspace) +
                 round_up(static_cast<size_t>(batch) * h->cfg.num_heads * h->cfg.d_v * act_bytes(h->cfg.act_dtype), 256);
   return map_cuda(launch_out_proj_umma(h, a, extra, stream));
@@ -451,6 +457,33 @@ int mla_last_device_error(mla_handle_t h, cudaStream_t stream) {
 int mla_set_wait_limit(mla_handle_t h, uint32_t limit) {
   if (h == nullptr) return MLA_ERR_INVALID_ARG;
   h->wait_limit = limit == 0 ? kDefaultWaitLimit : limit;
+  return MLA_OK;
+}
+
+static bool w_o_tileable(const mla_ctx* h) {
+  return h->cfg.d_model % 128 == 0 && (static_cast<long>(h->cfg.num_heads) * h->cfg.d_v) % 64 == 0;
+}
+
+int mla_pack_w_o(mla_handle_t h, const void* w_o, void* w_o_tiled, cudaStream_t stream) {
+  if (h == nullptr || w_o == nullptr || w_o_tiled == nullptr || w_o == w_o_tiled) return MLA_ERR_INVALID_ARG;
+  if (!w_o_tileable(h)) return MLA_ERR_UNSUPPORTED;
+  if (!aligned(w_o, 16) || !aligned(w_o_tiled, 16)) return MLA_ERR_ALIGNMENT;
+  if (!on_handle_device(h)) return MLA_ERR_INVALID_ARG;
+  return map_cuda(launch_pack_tiles(w_o, w_o_tiled, h->cfg.d_model,
+                                    static_cast<long>(h->cfg.num_heads) * h->cfg.d_v,
+                                    static_cast<int>(act_bytes(h->cfg.act_dtype)), stream));
+}
+
+int mla_set_w_o_layout(mla_handle_t h, int tiled) {
+  if (h == nullptr) return MLA_ERR_INVALID_ARG;
+  if (tiled && !w_o_tileable(h)) return MLA_ERR_UNSUPPORTED;
+  h->w_o_tiled = tiled ? 1 : 0;
+  return MLA_OK;
+}
+
+int mla_set_launch_overlap(mla_handle_t h, int enable) {
+  if (h == nullptr) return MLA_ERR_INVALID_ARG;
+  h->overlap = enable != 0 ? 1 : 0;
   return MLA_OK;
 }
 

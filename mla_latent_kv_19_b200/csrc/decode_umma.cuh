@@ -84,7 +84,6 @@ constexpr int kPBytes = kH * kTok * 2;                 // 16384
 constexpr int kPMsgBytes = kPBytes + kH * 4 + 16;      // P + alpha[128] + flag[4] = 16912
 constexpr int kPBufStride = 17 * 1024;                 // keeps every P tile 1024-byte aligned
 constexpr int kMaxTablePages = 512;                    // pages of a split kept in shared memory
-constexpr int kPrefetchPages = 0;                      // L2 prefetch distance ahead of the ring's loads (0: none)
 // e4m3 cache: a page is 64 rows x 576 code bytes, contiguous in the pool, plus
 // 64 fp32 per-token scales
 constexpr int kPageF8Bytes = kTok * kD;                // 36864
@@ -225,10 +224,6 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
   auto bar = [&](int i) -> uint32_t { return sb + kOffBar + 8u * static_cast<uint32_t>(i); };
   const uint32_t iters = a.wait_limit;
 
-  int bad_len = 0;
-  const Split sp = split_of(a, static_cast<int>(blockIdx.x >> 1), &bad_len);
-  if (bad_len && threadIdx.x == 0 && rank == 0) report_error(a.err, MLA_ERR_BAD_INDEX);
-
   auto fail = [&]() {
     misc[1] = 1u;
     report_error(a.err, MLA_ERR_TIMEOUT);
@@ -247,13 +242,8 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
   };
   auto drain = [&](uint32_t b_, uint32_t par) { ptx::mbar_wait<false>(b_, par, kDrainIters, kWaitNs); };
 
-  // this split's page table, kept in shared memory
-  int* table = reinterpret_cast<int*>(smem + (rank == 0 ? kOffTable0 : kOffTable1));
-  for (int t = threadIdx.x; t < min(sp.ntiles, kMaxTablePages); t += blockDim.x) {
-    const int pg = load_page(a, sp, t);
-    table[t] = pg;
-    if (pg < 0 && rank == 0) report_error(a.err, MLA_ERR_BAD_INDEX);
-  }
+  // set-up that reads none of the call's inputs runs before the wait for the
+  // previous kernel of the stream (programmatic dependent launch)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSlots; ++i) {
       ptx::mbar_init(bar(kFull + i), 1);
@@ -303,6 +293,20 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = misc[0];
 
+  grid_dep_wait();
+  grid_dep_trigger();
+  int bad_len = 0;
+  const Split sp = split_of(a, static_cast<int>(blockIdx.x >> 1), &bad_len);
+  if (bad_len && threadIdx.x == 0 && rank == 0) report_error(a.err, MLA_ERR_BAD_INDEX);
+  // this split's page table, kept in shared memory
+  int* table = reinterpret_cast<int*>(smem + (rank == 0 ? kOffTable0 : kOffTable1));
+  for (int t = threadIdx.x; t < min(sp.ntiles, kMaxTablePages); t += blockDim.x) {
+    const int pg = load_page(a, sp, t);
+    table[t] = pg;
+    if (pg < 0 && rank == 0) report_error(a.err, MLA_ERR_BAD_INDEX);
+  }
+  __syncthreads();
+
   if (rank == 0) {
     // =========================== CTA 0: scores and softmax ===========================
     // Slot use n = 0, 1 carries Q half n; use n >= 2 carries tile t = n - 2.
@@ -312,17 +316,6 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         // each as soon as the slot is free (its previous page's MMAs are done).
         if (!kFp8) ptx::prefetch_tmap(&kmap);
         ptx::prefetch_tmap(&qmap);
-        auto prefetch_page = [&](int t) {
-          if (kPrefetchPages == 0 || t >= sp.ntiles) return;
-          const long pg = max(page_at(a, sp, table, t), 0);
-          if (kFp8) {
-            ptx::prefetch_l2(static_cast<const uint8_t*>(a.cache) + pg * kPageF8Bytes, kPageF8Bytes);
-            ptx::prefetch_l2(a.cache_scale + pg * kTok, kScaleBytes);
-          } else {
-            ptx::prefetch_l2(static_cast<const uint8_t*>(a.cache) + pg * kSlotBytes, kSlotBytes);
-          }
-        };
-        for (int t = 0; t < kPrefetchPages; ++t) prefetch_page(t);
         const int total = kQLoads + sp.ntiles;
         int issued = 0;
         for (int n = 0; n < total; ++n) {
@@ -335,7 +328,6 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
           } else {
             const int t = n - kQLoads;
             const int pg = max(page_at(a, sp, table, t), 0);
-            prefetch_page(t + kPrefetchPages);
             if (kFp8) {
               // the page's codes (contiguous) into the slot's upper half, its scales
               // into scale-ring entry t % 6
@@ -920,15 +912,21 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
         if (sp.ntiles == 0) {
           for (int g = 8 * c0; g < 8 * c1; ++g) obase[g * kH] = make_float4(0.f, 0.f, 0.f, 0.f);
         } else {
+          // two 32-column blocks per TMEM round trip where registers allow (bf16)
+          constexpr int kPer = kFp8 ? 1 : 2;
 #pragma unroll 1
-          for (int c = c0; c < c1; ++c) {
-            uint32_t v[32];
-            ptx::tmem_ld32(tmem + lb + kColO + 32u * c, v);
+          for (int c = c0; c < c1; c += kPer) {
+            uint32_t v[kPer][32];
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) ptx::tmem_ld32(tmem + lb + kColO + 32u * (c + j), v[j]);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              obase[(8 * c + e) * kH] = make_float4(__uint_as_float(v[4 * e]) * inv, __uint_as_float(v[4 * e + 1]) * inv,
-                                                    __uint_as_float(v[4 * e + 2]) * inv, __uint_as_float(v[4 * e + 3]) * inv);
+            for (int j = 0; j < kPer; ++j)
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                obase[(8 * (c + j) + e) * kH] =
+                    make_float4(__uint_as_float(v[j][4 * e]) * inv, __uint_as_float(v[j][4 * e + 1]) * inv,
+                                __uint_as_float(v[j][4 * e + 2]) * inv, __uint_as_float(v[j][4 * e + 3]) * inv);
           }
         }
         ptx::tc_fence_before();

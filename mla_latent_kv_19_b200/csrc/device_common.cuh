@@ -21,6 +21,16 @@ template <> __device__ __forceinline__ __nv_bfloat16 cvt_out<__nv_bfloat16>(floa
   return __float2bfloat16_rn(x);
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the kernel issued before it on the stream is
+// still running.  grid_dep_wait() returns once that kernel has completed and
+// its writes are visible (a no-op for a normal launch); grid_dep_trigger()
+// lets the kernel issued after this one begin its launch.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Record the first device-side error of a handle (later ones are dropped).
 __device__ __forceinline__ void report_error(int* err, int code) {
   if (err != nullptr && *reinterpret_cast<volatile int*>(err) == 0) atomicCAS(err, 0, code);

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/mla.h"
 
 struct mla_ctx {
@@ -16,6 +18,8 @@ struct mla_ctx {
   float2* rope_cs;     // device [max_position][d_r/2] (cos, sin)
   int* err;            // device error word (0 = no error)
   uint32_t wait_limit; // bounded-wait iteration limit (0 = default)
+  int overlap;         // launch kernels as programmatic dependents of the previous one
+  int w_o_tiled;       // W_O arguments are tile-major (mla_pack_w_o)
 };
 
 namespace mla {
@@ -24,6 +28,25 @@ constexpr uint32_t kDefaultWaitLimit = 1u << 26;
 
 // Counts kernel launches (host side); read through mla_launch_count().
 void note_launches(int n);
+
+// Launch `k`; with `overlap`, as a programmatic dependent launch: the kernel may
+// begin while the previous kernel of the stream is still running, so it must
+// call grid_dep_wait() before it touches anything that kernel reads or writes.
+template <typename... P, typename... A>
+cudaError_t launch_kernel(bool overlap, void (*k)(P...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t s, A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = overlap ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k, std::forward<A>(args)...);
+}
 
 // Work description shared by the append kernels.
 struct AppendArgs {
@@ -44,6 +67,7 @@ struct AppendArgs {
   const float2* rope_cs;
   int* err;
   int32_t d_c, d_r, d_model, block_size, max_position;
+  int32_t overlap;      // programmatic dependent launch
 };
 
 struct AbsorbArgs {
@@ -78,6 +102,7 @@ struct CombineArgs {
   void* o_lat;                // [B, H, d_c] act dtype
   float* lse;                 // [B, H] or null
   int32_t batch, num_heads, d_c, num_splits;
+  int32_t overlap;            // programmatic dependent launch
 };
 
 struct OutProjArgs {
@@ -93,6 +118,7 @@ struct OutProjArgs {
   const float* comb_lse;     // [B, S, H]
   int32_t comb_splits;
   float* comb_lse_out;       // [B, H] or null
+  int32_t w_o_tiled;         // w_o is tile-major: [d_model/128][H*d_v/64][128][64]
 };
 
 // Launchers (return cudaGetLastError() of their launches).
@@ -103,5 +129,9 @@ cudaError_t launch_decode_generic(const DecodeArgs& a, int act_dtype, int cache_
                                   cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, int act_dtype, int num_sms, cudaStream_t s);
 cudaError_t launch_out_proj_generic(const OutProjArgs& a, int act_dtype, cudaStream_t s);
+// dst[r/128][c/64][r%128][c%64] = src[r][c] for a rows x cols matrix of
+// elem_bytes-wide elements (rows % 128 == 0, cols % 64 == 0).
+cudaError_t launch_pack_tiles(const void* src, void* dst, long rows, long cols, int elem_bytes,
+                              cudaStream_t s);
 
 }  // namespace mla

@@ -6,6 +6,8 @@
 //     configuration with H=8, d_c=64, d_r=16).
 //
 // Method: DeepSeek V2 MLA page (snabindia.com), sections 2.1-2.3.
+#include <algorithm>
+
 #include "device_common.cuh"
 
 namespace mla {
@@ -95,6 +97,8 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(AppendArgs a)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int D = a.d_c + a.d_r;
   const int t = blockIdx.x * kAppendWarps + warp;
+  grid_dep_wait();
+  grid_dep_trigger();
   if (t >= a.num_tokens) return;
   const int b = a.seq_idx ? a.seq_idx[t] : t;
   const int p = a.pos[t];
@@ -162,9 +166,9 @@ cudaError_t launch_append(const AppendArgs& a, int act_dtype, int cache_dtype, b
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  k<<<grid, block, smem, s>>>(a);
+  const cudaError_t e = launch_kernel(a.overlap != 0, k, grid, block, smem, s, a);
   note_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 // ---------------------------------------------------------------------------
@@ -437,6 +441,8 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
   const int b = blockIdx.x, c0 = blockIdx.y * kCols;
   const int S = a.num_splits, H = a.num_heads;
   const int h = threadIdx.x;                  // blockDim.x == 128 >= H
+  grid_dep_wait();
+  grid_dep_trigger();
   if (h < H) {
     const float* lp = a.lse_part + static_cast<long>(b) * S * H + h;
     float m = -INFINITY;
@@ -494,9 +500,9 @@ cudaError_t launch_combine_cols(const CombineArgs& a, int act_dtype, cudaStream_
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  k<<<grid, 128, smem, s>>>(a);
+  const cudaError_t e = launch_kernel(a.overlap != 0, k, grid, dim3(128), smem, s, a);
   note_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_combine(const CombineArgs& a, int act_dtype, int num_sms, cudaStream_t s) {
@@ -550,6 +556,12 @@ __global__ void __launch_bounds__(256) uv_generic_kernel(OutProjArgs a) {
   }
 }
 
+// Offset of W_O[m][k] (K columns) in the row-major or the tile-major layout.
+__device__ __forceinline__ long w_o_offset(int m, int k, int K, bool tiled) {
+  return tiled ? ((static_cast<long>(m >> 7) * (K >> 6) + (k >> 6)) << 13) + ((m & 127) << 6) + (k & 63)
+               : static_cast<long>(m) * K + k;
+}
+
 // grid ceil(d_model / 8); warp per output row m; K = H*d_v streamed in chunks of 256.
 template <typename T>
 __global__ void __launch_bounds__(256) wo_generic_kernel(OutProjArgs a) {
@@ -558,7 +570,8 @@ __global__ void __launch_bounds__(256) wo_generic_kernel(OutProjArgs a) {
   const int m = blockIdx.x * 8 + warp;
   const int K = a.num_heads * a.d_v;
   const T* o = reinterpret_cast<const T*>(a.o);
-  const T* w = reinterpret_cast<const T*>(a.w_o) + static_cast<long>(m) * K;
+  const T* w = reinterpret_cast<const T*>(a.w_o);
+  const bool tiled = a.w_o_tiled != 0;
   T* y = reinterpret_cast<T*>(a.y);
   for (int b0 = 0; b0 < a.batch; b0 += kOpBatch) {
     const int nb = min(kOpBatch, a.batch - b0);
@@ -579,7 +592,7 @@ __global__ void __launch_bounds__(256) wo_generic_kernel(OutProjArgs a) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int kk = k0 + 8 * lane + e;
-          const float wv = kk < K ? ld_f32(w, kk) : 0.f;
+          const float wv = kk < K ? ld_f32(w, w_o_offset(m, kk, K, tiled)) : 0.f;
 #pragma unroll
           for (int i = 0; i < kOpBatch; ++i) acc[i] += wv * os[i][e * 32 + lane];
         }
@@ -593,6 +606,36 @@ __global__ void __launch_bounds__(256) wo_generic_kernel(OutProjArgs a) {
       }
     }
   }
+}
+
+// One thread per 16-byte unit of the tile-major output, in its order (the
+// reads are 16-byte pieces of 128-byte row segments).
+template <int kElem>
+__global__ void __launch_bounds__(256) pack_tiles_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                         long rows, long cols) {
+  constexpr int kPerUnit = 16 / kElem;                // elements per 16-byte unit
+  constexpr int kUnitsPerRow = 64 / kPerUnit;         // units per 64-column tile row
+  const long units = rows * cols / kPerUnit;
+  const long ctiles = cols / 64;
+  for (long u = blockIdx.x * 256L + threadIdx.x; u < units; u += gridDim.x * 256L) {
+    const long e = u % kUnitsPerRow, r = (u / kUnitsPerRow) % 128, tile = u / (kUnitsPerRow * 128);
+    const long rt = tile / ctiles, ct = tile % ctiles;
+    dst[u] = src[((rt * 128 + r) * cols + ct * 64) / kPerUnit + e];
+  }
+}
+
+cudaError_t launch_pack_tiles(const void* src, void* dst, long rows, long cols, int elem_bytes,
+                              cudaStream_t s) {
+  if (rows % 128 != 0 || cols % 64 != 0 || (elem_bytes != 2 && elem_bytes != 4)) return cudaErrorInvalidValue;
+  if (rows == 0 || cols == 0) return cudaSuccess;
+  const long units = rows * cols * elem_bytes / 16;
+  const dim3 grid(static_cast<unsigned>(std::min<long>((units + 255) / 256, 4096)));
+  if (elem_bytes == 2)
+    pack_tiles_kernel<2><<<grid, 256, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), rows, cols);
+  else
+    pack_tiles_kernel<4><<<grid, 256, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), rows, cols);
+  note_launches(1);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_out_proj_generic(const OutProjArgs& a, int act_dtype, cudaStream_t s) {

@@ -32,19 +32,24 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // column chunk), so that one box of box_rows x chunks lands in shared memory
 // chunk-major: [chunk][row][128 bytes], 128-byte swizzled -- the UMMA K-major
 // (and, for V, MN-major) operand layout.
-cudaError_t make_map_rows_chunked(CUtensorMap* map, const void* base, uint64_t rows,
-                                  uint64_t row_bytes, uint32_t chunks, uint32_t box_rows,
-                                  uint32_t box_chunks) {
+cudaError_t make_map_3d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t row_bytes,
+                        uint64_t chunks, uint64_t chunk_bytes, uint32_t box_rows, uint32_t box_chunks) {
   auto fn = encode_fn();
   if (fn == nullptr) return cudaErrorNotSupported;
   const cuuint64_t dims[3] = {64, rows, chunks};
-  const cuuint64_t strides[2] = {row_bytes, 128};
+  const cuuint64_t strides[2] = {row_bytes, chunk_bytes};
   const cuuint32_t box[3] = {64, box_rows, box_chunks};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_map_rows_chunked(CUtensorMap* map, const void* base, uint64_t rows,
+                                  uint64_t row_bytes, uint32_t chunks, uint32_t box_rows,
+                                  uint32_t box_chunks) {
+  return make_map_3d(map, base, rows, row_bytes, chunks, 128, box_rows, box_chunks);
 }
 
 }  // namespace
@@ -64,7 +69,7 @@ namespace {
 
 template <bool kFp8>
 cudaError_t launch_decode_kernel(const CUtensorMap& kmap, const CUtensorMap& vmap, const CUtensorMap& qmap,
-                                 const DecodeArgs& a, unsigned ctas, cudaStream_t s) {
+                                 const DecodeArgs& a, unsigned ctas, bool overlap, cudaStream_t s) {
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
@@ -72,8 +77,8 @@ cudaError_t launch_decode_kernel(const CUtensorMap& kmap, const CUtensorMap& vma
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  dec::decode_umma_kernel<kFp8><<<dim3(ctas), dec::threads<kFp8>(), dec::kSmemBytes, s>>>(kmap, vmap, qmap, a);
-  return cudaGetLastError();
+  return launch_kernel(overlap, dec::decode_umma_kernel<kFp8>, dim3(ctas), dim3(dec::threads<kFp8>()),
+                       dec::kSmemBytes, s, kmap, vmap, qmap, a);
 }
 
 }  // namespace
@@ -101,8 +106,9 @@ cudaError_t launch_decode_umma(const mla_ctx* h, const DecodeArgs& a, cudaStream
   if (e != cudaSuccess) return e;
   const long ctas = 2L * a.batch * a.num_splits;
   if (ctas > 0x7fffffffL) return cudaErrorInvalidValue;
-  e = fp8 ? launch_decode_kernel<true>(kmap, vmap, qmap, a, static_cast<unsigned>(ctas), s)
-          : launch_decode_kernel<false>(kmap, vmap, qmap, a, static_cast<unsigned>(ctas), s);
+  const bool ov = h->overlap != 0;
+  e = fp8 ? launch_decode_kernel<true>(kmap, vmap, qmap, a, static_cast<unsigned>(ctas), ov, s)
+          : launch_decode_kernel<false>(kmap, vmap, qmap, a, static_cast<unsigned>(ctas), ov, s);
   if (e == cudaSuccess) note_launches(1);
   return e;
 }
@@ -113,7 +119,21 @@ cudaError_t launch_decode_umma(const mla_ctx* h, const DecodeArgs& a, cudaStream
 
 namespace {
 
-constexpr int kOProjSplits = 3;      // K split of W_O: 40 row tiles x 3 = 120 CTAs, one per SM
+constexpr int kOProjSplits = 3;      // K split of W_O when stream-K does not apply
+
+// How W_O is split over the GPU: stream-K, one CTA per SM, each CTA taking an
+// equal run of the (M tile, box of kcs K chunks) stages.
+struct WoPlan {
+  int kcs;      // K chunks per stage (box depth)
+  int stages;
+  int box;      // stages per M tile
+  int units;    // M tiles x box
+  int g;        // CTAs
+  int slots;    // partial tiles per CTA (M tiles one run can touch)
+  bool stream_k;
+};
+
+int tmem_block_cols(int n) { return n <= 32 ? 32 : (n <= 64 ? 64 : (n <= 128 ? 128 : 256)); }
 
 int padded_n(int batch) { return (batch + 15) / 16 * 16; }
 
@@ -153,7 +173,7 @@ int gemm_tmem_cols(const gemm::Params& p) {
 
 template <bool kAMn, gemm::Epi kEpi>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tx, gemm::Params p, dim3 grid,
-                        cudaStream_t s) {
+                        bool overlap, cudaStream_t s) {
   if (gemm_tmem_cols(p) > 512) return cudaErrorInvalidValue;     // TMEM holds 512 columns
   // as many stages as requested that fit in shared memory (larger batches: fewer)
   while (p.stages > 2 && gemm_smem_bytes(p) > 232448) --p.stages;
@@ -161,9 +181,9 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tx, gemm::Para
   if (smem > 232448) return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem_limit(gemm::gemm_wt_kernel<kAMn, kEpi>, smem);
   if (e != cudaSuccess) return e;
-  gemm::gemm_wt_kernel<kAMn, kEpi><<<grid, 256, smem, s>>>(ta, tx, p);
+  e = launch_kernel(overlap, gemm::gemm_wt_kernel<kAMn, kEpi>, grid, dim3(256), smem, s, ta, tx, p);
   note_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 bool v2_bf16(const mla_ctx* h) {
@@ -218,12 +238,50 @@ cudaError_t launch_absorb_umma(const mla_ctx* h, const AbsorbArgs& a, cudaStream
   p.err = a.err;
   p.wait_limit = h->wait_limit;
   const int ctas_per_head = (a.d_c / gemm::kM) / p.mt_per_cta;
-  return launch_gemm<true, gemm::Epi::kAbsorb>(ta, tx, p, dim3(H * ctas_per_head, 1), s);
+  return launch_gemm<true, gemm::Epi::kAbsorb>(ta, tx, p, dim3(H * ctas_per_head, 1), h->overlap != 0, s);
 }
 
 bool umma_out_proj_supported(const mla_ctx* h, int batch) {
   return v2_bf16(h) && batch >= 1 && batch <= 256;
 }
+
+namespace {
+
+WoPlan wo_plan(const mla_ctx* h, int batch) {
+  const int n = padded_n(batch);
+  WoPlan w{};
+  auto fits = [&](int kcs, int stages) {
+    return static_cast<long>(stages) * (gemm::kM + n) * gemm::kKc * 2 * kcs + 8 * (2 * stages + 4) + 16 + 1024 <=
+           232448;
+  };
+  // (measured) the row-major weight streams fastest as 64 KB boxes in two stages,
+  // the tile-major one as 48 KB boxes in three; larger batches fall back to 32 KB
+  // boxes in as many stages as fit
+  if (h->w_o_tiled && fits(3, 3)) {
+    w.kcs = 3;
+    w.stages = 3;
+  } else if (fits(4, 2)) {
+    w.kcs = 4;
+    w.stages = 2;
+  } else {
+    w.kcs = 2;
+    w.stages = 5;
+  }
+  const int k_chunks = h->cfg.num_heads * h->cfg.d_v / gemm::kKc;
+  const int m_tiles = h->cfg.d_model / gemm::kM;
+  w.box = (k_chunks + w.kcs - 1) / w.kcs;
+  w.units = m_tiles * w.box;
+  w.g = std::max(1, std::min(h->num_sms, w.units));
+  const int run = (w.units + w.g - 1) / w.g;
+  w.slots = std::min((run + w.box - 1) / w.box + 1, m_tiles);
+  int cols = 32;
+  while (cols < tmem_block_cols(n) * w.slots) cols <<= 1;
+  // (the reduce kernel locates partials in 32-bit arithmetic)
+  w.stream_k = cols <= 512 && static_cast<long>(w.units) * w.g < (1L << 31);
+  return w;
+}
+
+}  // namespace
 
 bool umma_combine_out_proj_supported(const mla_ctx* h, int batch, int num_splits) {
   if (!umma_out_proj_supported(h, batch) || num_splits < 1 || h->cfg.num_heads > 128) return false;
@@ -236,7 +294,10 @@ bool umma_combine_out_proj_supported(const mla_ctx* h, int batch, int num_splits
 
 size_t umma_out_proj_extra_workspace(const mla_ctx* h, int batch) {
   if (!umma_out_proj_supported(h, batch)) return 0;
-  return static_cast<size_t>(kOProjSplits) * batch * h->cfg.d_model * sizeof(float) + 256;
+  const WoPlan w = wo_plan(h, batch);
+  const size_t ks = static_cast<size_t>(kOProjSplits) * batch * h->cfg.d_model * sizeof(float);
+  const size_t sk = static_cast<size_t>(w.g) * w.slots * batch * gemm::kM * sizeof(float);
+  return (w.stream_k ? sk : ks) + 256;
 }
 
 cudaError_t launch_out_proj_umma(const mla_ctx* h, const OutProjArgs& a, void* extra,
@@ -284,45 +345,71 @@ cudaError_t launch_out_proj_umma(const mla_ctx* h, const OutProjArgs& a, void* e
     }
     p.err = h->err;
     p.wait_limit = h->wait_limit;
-    e = launch_gemm<false, gemm::Epi::kStoreBf16T>(ta, tx, p, dim3(H, 1), s);
+    e = launch_gemm<false, gemm::Epi::kStoreBf16T>(ta, tx, p, dim3(H, 1), h->overlap != 0, s);
     if (e != cudaSuccess) return e;
   }
-  // partial[s][b][m] = sum over this split's K of W_O[m][k] o[b][k]
+  // fp32 partials of y: stream-K slots, or one [b][m] block per K split
   float* part = static_cast<float*>(extra);
+  const WoPlan w = wo_plan(h, a.batch);
   {
-    // 64 KB weight boxes in two stages stream faster than smaller boxes in more
-    // stages (measured); larger batches fall back to 32 KB boxes to fit
-    const int kcs = 2 * (gemm::kM + n) * gemm::kKc * 2 * 4 + 4096 <= 232448 ? 4 : 2;
     CUtensorMap ta, tx;
-    cudaError_t e = make_map_rows_chunked(&ta, a.w_o, a.d_model, kdim * 2, kdim / gemm::kKc, gemm::kM, kcs);
+    // row-major: (64 columns, row, chunk); tile-major: (64 columns, row of the
+    // tile, tile * k_chunks + chunk), a 16 KB tile per 64-column chunk
+    cudaError_t e =
+        a.w_o_tiled ? make_map_3d(&ta, a.w_o, gemm::kM, 128, static_cast<uint64_t>(a.d_model / gemm::kM) * (kdim / gemm::kKc),
+                                  gemm::kM * 128, gemm::kM, w.kcs)
+                    : make_map_rows_chunked(&ta, a.w_o, a.d_model, kdim * 2, kdim / gemm::kKc, gemm::kM, w.kcs);
     if (e != cudaSuccess) return e;
-    e = make_map_rows_chunked(&tx, a.o, a.batch, kdim * 2, kdim / gemm::kKc, n, kcs);
+    e = make_map_rows_chunked(&tx, a.o, a.batch, kdim * 2, kdim / gemm::kKc, n, w.kcs);
     if (e != cudaSuccess) return e;
     gemm::Params p{};
     p.n = n;
     p.batch = a.batch;
     p.k_chunks = static_cast<int>(kdim / gemm::kKc);
-    p.k_split = kOProjSplits;
     p.m_per_group = a.d_model;
-    p.mt_per_cta = 1;
-    p.kcs = kcs;
+    p.kcs = w.kcs;
     p.a_row_group = 0;
     p.x_col_group = 0;
-    p.stages = kcs == 4 ? 2 : 5;
+    p.stages = w.stages;
+    p.a_tiled = a.w_o_tiled;
     p.out = part;
-    p.out_ld = a.d_model;
     p.out_group = 0;
-    p.out_split = static_cast<long>(a.batch) * a.d_model;
     p.err = h->err;
     p.wait_limit = h->wait_limit;
-    e = launch_gemm<false, gemm::Epi::kPartialF32>(ta, tx, p, dim3(a.d_model / gemm::kM, kOProjSplits), s);
+    dim3 grid;
+    if (w.stream_k) {
+      // partial[c * slots + t][b][r] for the t-th M tile of CTA c
+      p.k_split = 1;
+      p.mt_per_cta = w.slots;
+      p.sk_units = w.units;
+      p.sk_box = w.box;
+      p.out_ld = gemm::kM;
+      p.out_split = static_cast<long>(a.batch) * gemm::kM;
+      grid = dim3(w.g, 1);
+    } else {
+      // partial[s][b][m] = sum over split s's K of W_O[m][k] o[b][k]
+      p.k_split = kOProjSplits;
+      p.mt_per_cta = 1;
+      p.out_ld = a.d_model;
+      p.out_split = static_cast<long>(a.batch) * a.d_model;
+      grid = dim3(a.d_model / gemm::kM, kOProjSplits);
+    }
+    e = launch_gemm<false, gemm::Epi::kPartialF32>(ta, tx, p, grid, h->overlap != 0, s);
     if (e != cudaSuccess) return e;
   }
   const long count = static_cast<long>(a.batch) * a.d_model;
-  gemm::reduce_splits_kernel<<<static_cast<unsigned>(std::min<long>((count + 255) / 256, 1184)), 256, 0, s>>>(
-      part, static_cast<__nv_bfloat16*>(a.y), kOProjSplits, count);
+  const dim3 rgrid(static_cast<unsigned>(std::min<long>((count + 255) / 256, 1184)));
+  cudaError_t e;
+  if (w.stream_k) {
+    e = launch_kernel(h->overlap != 0, gemm::reduce_stream_k_kernel,
+                      dim3(a.d_model / gemm::kM, (a.batch + 1) / 2), dim3(256), 0, s, part,
+                      static_cast<__nv_bfloat16*>(a.y), a.batch, a.d_model, w.units, w.box, w.g, w.slots);
+  } else {
+    e = launch_kernel(h->overlap != 0, gemm::reduce_splits_kernel, rgrid, dim3(256), 0, s, part,
+                      static_cast<__nv_bfloat16*>(a.y), kOProjSplits, count);
+  }
   note_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace mla

@@ -18,7 +18,8 @@ import torch
 
 from . import (Handle, mla_absorb_q, mla_cache_append, mla_combine_out_proj, mla_decode_auto_splits,
                mla_decode_combine, mla_decode_partial, mla_decode_workspace_bytes,
-               mla_kv_project_append, mla_out_proj, mla_out_proj_workspace_bytes)
+               mla_kv_project_append, mla_out_proj, mla_out_proj_workspace_bytes, mla_pack_w_o,
+               mla_set_launch_overlap, mla_set_w_o_layout)
 
 BLOCK_SIZE = 64
 
@@ -41,7 +42,13 @@ def softmax_scale(d_nope: int, d_r: int) -> float:
 
 
 class DecodeStep:
-    def __init__(self, wl, device="cuda", num_splits: int = 0, max_position: Optional[int] = None):
+    def __init__(self, wl, device="cuda", num_splits: int = 0, max_position: Optional[int] = None,
+                 overlap: bool = False, w_o_tiled: bool = True):
+        """overlap: launch each kernel as a programmatic dependent of the one
+        before it (its set-up and first weight loads overlap that kernel's end);
+        the step never writes a weight, which is what that asks of the caller.
+        w_o_tiled: keep W_O in the library's tile-major order (packed once here)
+        where the shape allows; ``self.w_o`` is then that copy."""
         d = wl.dims
         self.wl = wl
         self.device = torch.device(device)
@@ -60,6 +67,7 @@ class DecodeStep:
                             act_dtype=wl.act_dtype, cache_dtype=wl.cache_dtype,
                             softmax_scale=softmax_scale(self.d_nope, self.d_r),
                             rope_base=wl.rope_base, max_position=max_position)
+        mla_set_launch_overlap(self.h, overlap)
         dev = self.device
         act = torch.float32 if wl.act_dtype == "fp32" else torch.bfloat16
         self.act = act
@@ -80,6 +88,13 @@ class DecodeStep:
         self.w_uk = to_device(wl.w_uk, dev)
         self.w_uv = to_device(wl.w_uv, dev)
         self.w_o = to_device(wl.w_o, dev)
+        self.w_o_tiled = w_o_tiled and self.d_model % 128 == 0 and (self.H * self.d_v) % 64 == 0
+        if self.w_o_tiled:
+            packed = torch.empty_like(self.w_o)
+            mla_pack_w_o(self.h, self.w_o, packed)
+            torch.cuda.synchronize(dev)
+            self.w_o = packed
+            mla_set_w_o_layout(self.h, True)
         if self.tiny:
             self.w_dkv = to_device(wl.w_dkv, dev)
             self.w_kr = to_device(wl.w_kr, dev)
@@ -101,6 +116,10 @@ class DecodeStep:
         self.set_splits(num_splits)
         nb = mla_out_proj_workspace_bytes(self.h, B)
         self.op_ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
+        # run(): the append on a side stream beside the absorb
+        self.side = torch.cuda.Stream(device=dev)
+        self._fork = torch.cuda.Event()
+        self._join = torch.cuda.Event()
         self.prefill()
 
     def set_splits(self, num_splits: int) -> None:
@@ -166,6 +185,21 @@ class DecodeStep:
                 ("combine_out_proj", self.combine_out_proj)]
 
     def run(self, stream=None) -> None:
+        """One decode step.  The append and the absorbed query are independent
+        (one writes the cache, the other reads q and W_UK), so the append runs on
+        a side stream beside the absorb; the decode waits for both."""
+        main = stream if stream is not None else torch.cuda.current_stream(self.device)
+        self._fork.record(main)
+        self.side.wait_event(self._fork)
+        self.append(self.side)
+        self._join.record(self.side)
+        self.absorb(main)
+        main.wait_event(self._join)
+        self.decode_partial(main)
+        self.combine_out_proj(main)
+
+    def run_in_order(self, stream=None) -> None:
+        """The step's calls one after another on one stream."""
         for _, fn in self.stages():
             fn(stream)
 

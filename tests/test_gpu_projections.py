@@ -105,3 +105,62 @@ def test_fused_merge_out_proj_equals_the_two_calls(name, kw, splits):
     g = {k: v.float().cpu().numpy() for k, v in out.items()}
     for k in ("o_lat", "lse", "y"):
         assert_close(k, g[k], r[k])
+
+
+@pytest.mark.parametrize("name", ["v2_b32_l2048", "tiny_fp32"])
+def test_pack_w_o_is_the_tile_major_relayout(name):
+    """mla_pack_w_o writes W_O[m][k] to [m/128][k/64][m%128][k%64], bit for bit
+    (bf16 and fp32 elements)."""
+    from mla_latent_kv_19_b200 import mla_pack_w_o
+    from mla_latent_kv_19_b200.step import to_device
+    wl = workloads.make(name, batch=1, context=64)
+    h = _handle_for(wl)
+    w = to_device(wl.w_o, "cuda")
+    t = torch.full_like(w, float("nan"))
+    mla_pack_w_o(h, w, t)
+    torch.cuda.synchronize()
+    h.close()
+    M, K = wl.w_o.shape
+    want = wl.w_o.reshape(M // 128, 128, K // 64, 64).transpose(0, 2, 1, 3).reshape(M, K)
+    got = t.view(torch.int16).cpu().numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.cpu().numpy()
+    np.testing.assert_array_equal(got, want)
+
+
+def _handle_for(wl):
+    from mla_latent_kv_19_b200 import Handle
+    from mla_latent_kv_19_b200.step import softmax_scale
+    d = wl.dims
+    return Handle(num_heads=d["num_heads"], d_c=d["d_c"], d_r=d["d_r"], d_nope=d["d_nope"], d_v=d["d_v"],
+                  d_model=d["d_model"], act_dtype=wl.act_dtype, cache_dtype=wl.cache_dtype,
+                  softmax_scale=softmax_scale(d["d_nope"], d["d_r"]), max_position=4096)
+
+
+@pytest.mark.parametrize("batch", BATCHES + [300])
+def test_out_proj_with_tile_major_w_o_against_oracle(batch):
+    """The output projection reading the tile-major W_O (tensor-core path up to
+    256 tokens, CUDA-core path beyond) matches the oracle."""
+    from mla_latent_kv_19_b200 import (mla_last_device_error, mla_out_proj, mla_out_proj_workspace_bytes,
+                                       mla_pack_w_o, mla_set_w_o_layout)
+    from mla_latent_kv_19_b200.step import to_device
+    wl = workloads.make("v2_b32_l2048", batch=1, context=64)
+    d = wl.dims
+    rng = np.random.default_rng(3000 + batch)
+    o_lat = workloads.f32_to_bf16_bits(
+        rng.standard_normal((batch, d["num_heads"], d["d_c"])).astype(np.float32))
+    h = _handle(d)
+    w_o = to_device(wl.w_o, "cuda")
+    w_t = torch.empty_like(w_o)
+    mla_pack_w_o(h, w_o, w_t)
+    del w_o
+    mla_set_w_o_layout(h, True)
+    ws = torch.empty(max(mla_out_proj_workspace_bytes(h, batch), 256), dtype=torch.uint8, device="cuda")
+    y = torch.empty(batch, d["d_model"], dtype=torch.bfloat16, device="cuda")
+    o = torch.empty(batch, d["num_heads"], d["d_v"], dtype=torch.bfloat16, device="cuda")
+    mla_out_proj(h, to_device(o_lat, "cuda"), to_device(wl.w_uv, "cuda"), w_t, ws, y, o)
+    assert mla_last_device_error(h) == 0
+    g_y, g_o = y.float().cpu().numpy(), o.float().cpu().numpy()
+    h.close()
+    r_o = oracle.up_project_out(workloads.bf16_to_f64(o_lat), wl.to_f64(wl.w_uv))
+    r_y = oracle.out_project(r_o, wl.to_f64(wl.w_o))
+    assert_close("o", g_o, r_o)
+    assert_close("y", g_y, r_y)
