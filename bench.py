@@ -390,10 +390,11 @@ def main():
         "kernels": kernels,
         "roofline": roof,
         "gpu_launches": int(launches),
-        "graphs": "each timed step is one replay of a CUDA graph of the step's C-ABI calls (kernels "
-                  "launched as programmatic dependents of the one before), timed by events at its two "
-                  "ends; the per-stage times come from a second graph with events between the stages, "
-                  "replayed after it; e2e replays the step graph",
+        "graphs": "each timed step is one replay of a CUDA graph of the step's C-ABI calls (append on a "
+                  "side stream beside the absorb" + ("; kernels launched as programmatic dependents of the "
+                  "one before" if args.overlap else "") + "), timed by events at its two ends; the per-stage "
+                  "times come from a second graph with events between the stages, replayed after it; e2e "
+                  "replays the step graph",
         "clocks": clk,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_s * 1e3},
