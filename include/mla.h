@@ -64,7 +64,8 @@ typedef enum {
   MLA_ERR_LAUNCH = -5,       /* a kernel launch failed (cudaGetLastError)          */
   MLA_ERR_BAD_INDEX = -6,    /* device: page-table entry or position out of range  */
   MLA_ERR_TIMEOUT = -7,      /* device: a bounded wait gave up                     */
-  MLA_ERR_CUDA = -8          /* another CUDA runtime error                         */
+  MLA_ERR_CUDA = -8,         /* another CUDA runtime error                         */
+  MLA_ERR_RANGE = -9         /* device: a value beyond the range of an fp16 split partial */
 } mla_status_t;
 
 typedef enum { MLA_BF16 = 0, MLA_FP8_E4M3 = 1, MLA_FP32 = 2 } mla_dtype_t;
@@ -190,10 +191,14 @@ MLA_API int mla_decode(mla_handle_t h, const void* q_lat, const void* cache, con
 /* The two halves of mla_decode, for callers that time or schedule them
  * separately.  mla_decode_partial writes the workspace; mla_decode_combine
  * reads it (same batch / num_splits / max_seq_len) and writes o_lat and lse.
- * Workspace layout (fp32): o_part [batch][S][d_c/4][H][4] (groups of four
- * latent columns, heads next: o_part[b][s][c/4][h][c%4]) followed, at the next
- * 256-byte boundary, by lse_part [batch][S][H]; an empty range stores
- * lse_part = -inf, o_part = 0. */
+ * Workspace layout: o_part, then at the next 256-byte boundary lse_part fp32
+ * [batch][S][H].  o_part holds each split's normalised partial output in
+ * 16-byte groups of latent columns, heads next: with bf16 activations fp16
+ * [batch][S][d_c/8][H][8] (o_part[b][s][c/8][h][c%8]), with fp32 activations
+ * fp32 [batch][S][d_c/4][H][4].  An empty range stores lse_part = -inf,
+ * o_part = 0.  An fp16 partial holds |value| <= 65504: a larger latent
+ * output (only from cache values of that size) records MLA_ERR_RANGE in the
+ * device error word. */
 MLA_API int mla_decode_partial(mla_handle_t h, const void* q_lat, const void* cache,
                        const float* cache_scale, int32_t num_blocks, const int32_t* block_table,
                        int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t batch,

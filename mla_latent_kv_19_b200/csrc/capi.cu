@@ -40,9 +40,17 @@ int resolve_splits(const mla_ctx* h, int32_t batch, int32_t max_seq_len, int32_t
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Bytes of one split partial value: fp16 with bf16 activations, fp32 with fp32.
+size_t part_elem_bytes(const mla_ctx* h) { return h->cfg.act_dtype == MLA_FP32 ? 4 : 2; }
+
+// Bytes of o_part for `parts` (sequence, split, head) rows, rounded to 256.
+size_t opart_bytes(const mla_ctx* h, size_t parts) {
+  return round_up(parts * h->cfg.d_c * part_elem_bytes(h), 256);
+}
+
 size_t decode_ws_bytes(const mla_ctx* h, int32_t batch, int32_t splits) {
   const size_t parts = static_cast<size_t>(batch) * splits * h->cfg.num_heads;
-  return round_up(parts * h->cfg.d_c * sizeof(float), 256) + round_up(parts * sizeof(float), 256);
+  return opart_bytes(h, parts) + round_up(parts * sizeof(float), 256);
 }
 
 }  // namespace
@@ -66,6 +74,7 @@ const char* mla_status_string(int s) {
     case MLA_ERR_BAD_INDEX: return "MLA_ERR_BAD_INDEX";
     case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT";
     case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_RANGE: return "MLA_ERR_RANGE";
     default: return "MLA_ERR_UNKNOWN";
   }
 }
@@ -303,9 +312,8 @@ int mla_decode_partial(mla_handle_t h, const void* q_lat, const void* cache,
   a.block_table = block_table;
   a.seq_lens = seq_lens;
   const size_t parts = static_cast<size_t>(batch) * S * h->cfg.num_heads;
-  a.o_part = static_cast<float*>(workspace);
-  a.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                        round_up(parts * h->cfg.d_c * sizeof(float), 256));
+  a.o_part = workspace;
+  a.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + opart_bytes(h, parts));
   a.err = h->err;
   a.batch = batch;
   a.num_heads = h->cfg.num_heads;
@@ -332,9 +340,8 @@ int mla_decode_combine(mla_handle_t h, int32_t batch, int32_t max_seq_len, int32
   if (!aligned(o_lat, 16) || (lse && !aligned(lse, 4))) return MLA_ERR_ALIGNMENT;
   CombineArgs a{};
   const size_t parts = static_cast<size_t>(batch) * S * h->cfg.num_heads;
-  a.o_part = static_cast<const float*>(workspace);
-  a.lse_part = reinterpret_cast<const float*>(static_cast<const char*>(workspace) +
-                                              round_up(parts * h->cfg.d_c * sizeof(float), 256));
+  a.o_part = workspace;
+  a.lse_part = reinterpret_cast<const float*>(static_cast<const char*>(workspace) + opart_bytes(h, parts));
   a.o_lat = o_lat;
   a.lse = lse;
   a.batch = batch;
@@ -433,9 +440,8 @@ int mla_combine_out_proj(mla_handle_t h, int32_t batch, int32_t max_seq_len, int
   a.d_c = h->cfg.d_c;
   a.d_v = h->cfg.d_v;
   a.d_model = h->cfg.d_model;
-  a.comb_opart = static_cast<const float*>(workspace);
-  a.comb_lse = reinterpret_cast<const float*>(static_cast<const char*>(workspace) +
-                                              round_up(parts * h->cfg.d_c * sizeof(float), 256));
+  a.comb_opart = static_cast<const __half*>(workspace);
+  a.comb_lse = reinterpret_cast<const float*>(static_cast<const char*>(workspace) + opart_bytes(h, parts));
   a.comb_splits = S;
   a.comb_lse_out = lse;
   a.w_o_tiled = h->w_o_tiled;

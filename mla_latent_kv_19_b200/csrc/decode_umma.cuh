@@ -901,16 +901,17 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
       bool ok = wait_local(bar(kOFull), 0);
       ok = ok && wait_remote(bar(kFin), 0);
       ok = __all_sync(0xffffffffu, ok);
-      // o_part[b][split][c/4][h][c%4]: per group of four columns the 32 lanes store
-      // 32 consecutive heads' float4s (512 contiguous bytes)
-      float4* obase = reinterpret_cast<float4*>(a.o_part) +
-                      (static_cast<long>(sp.b) * a.num_splits + sp.split) * (kDc / 4) * kH + r;
+      // o_part[b][split][c/8][h][c%8] in fp16: per group of eight columns the 32
+      // lanes store 32 consecutive heads' 16 bytes (512 contiguous bytes)
+      uint4* obase = reinterpret_cast<uint4*>(a.o_part) +
+                     (static_cast<long>(sp.b) * a.num_splits + sp.split) * (kDc / 8) * kH + r;
       if (ok) {
         ptx::tc_fence_after();
         const float lsum = reinterpret_cast<const volatile float*>(smem + kOffLfin)[r];
         const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+        float big = 0.f;
         if (sp.ntiles == 0) {
-          for (int g = 8 * c0; g < 8 * c1; ++g) obase[g * kH] = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int g = 4 * c0; g < 4 * c1; ++g) obase[g * kH] = make_uint4(0u, 0u, 0u, 0u);
         } else {
           // two 32-column blocks per TMEM round trip where registers allow (bf16)
           constexpr int kPer = kFp8 ? 1 : 2;
@@ -923,12 +924,23 @@ __global__ void __launch_bounds__(threads<kFp8>(), 1) __cluster_dims__(2, 1, 1)
 #pragma unroll
             for (int j = 0; j < kPer; ++j)
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                obase[(8 * (c + j) + e) * kH] =
-                    make_float4(__uint_as_float(v[j][4 * e]) * inv, __uint_as_float(v[j][4 * e + 1]) * inv,
-                                __uint_as_float(v[j][4 * e + 2]) * inv, __uint_as_float(v[j][4 * e + 3]) * inv);
+              for (int e = 0; e < 4; ++e) {
+                uint32_t hw[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const float x0 = __uint_as_float(v[j][8 * e + 2 * k]) * inv;
+                  const float x1 = __uint_as_float(v[j][8 * e + 2 * k + 1]) * inv;
+                  big = fmaxf(big, fmaxf(fabsf(x0), fabsf(x1)));
+                  const __half2 hh = __floats2half2_rn(x0, x1);
+                  hw[k] = *reinterpret_cast<const uint32_t*>(&hh);
+                }
+                obase[(4 * (c + j) + e) * kH] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              }
           }
         }
+        // fp16 holds |x| <= 65504 (the largest finite value); beyond it the
+        // partial would be infinite
+        if (!(big <= 65504.f)) report_error(a.err, MLA_ERR_RANGE);
         ptx::tc_fence_before();
       }
     } else if (kFp8 && warp >= 8) {

@@ -69,7 +69,7 @@ struct Params {
   // W_UV fed straight from split-KV partials: the resident X slice o_lat[:, h, :]
   // is merged in the kernel (log-sum-exp weights, as the merge kernel computes
   // them) instead of being loaded; comb_splits = 0 turns this off
-  const float* comb_opart;     // o_part [batch][S][d_c/4][H][4]
+  const __half* comb_opart;    // o_part fp16 [batch][S][d_c/8][H][8]
   const float* comb_lse;       // lse_part [batch][S][H]
   int comb_splits;             // S
   __nv_bfloat16* comb_olat;    // optional: o_lat [batch][H][d_c] is written too
@@ -301,12 +301,12 @@ __global__ void __launch_bounds__(256, 1)
     ptx::mbar_arrive(wready);
     const bool wok = wait(wready, 0);
     if (wok) {
-      const int dq = p.d_c / 4;
-      const float4* op = reinterpret_cast<const float4*>(p.comb_opart);
+      const int d8 = p.d_c / 8;
+      const uint4* op = reinterpret_cast<const uint4*>(p.comb_opart);   // 8 fp16 per head and group
       // 16-byte unit u: row b, K chunk k, unit v (columns 64k + 8v .. +7).  A
       // thread takes kU units at a time and loads two splits of all of them
-      // before it accumulates, so that 16 loads are in flight, not 2
-      constexpr int kU = 4;
+      // before it accumulates, so that 16 loads are in flight, not 1
+      constexpr int kU = 8;
       const int total = p.n * 8 * p.x_chunks;
       for (int ub = ct; ub < total; ub += kCombThreads * kU) {
         int bq[kU];
@@ -317,28 +317,29 @@ __global__ void __launch_bounds__(256, 1)
           const int u = ub + q * kCombThreads;
           const int b = u / (8 * p.x_chunks), k = (u / 8) % p.x_chunks, v = u % 8;
           bq[q] = u < total ? b : -1;
-          base[q] = (static_cast<long>(b) * S * dq + (64 * k + 8 * v) / 4) * H + h;
+          base[q] = (static_cast<long>(b) * S * d8 + 8 * k + v) * H + h;
 #pragma unroll
           for (int e = 0; e < 8; ++e) acc[q][e] = 0.f;
         }
         for (int sp = 0; sp < S; sp += 2) {
-          float4 x[2][kU][2];
+          uint4 x[2][kU];
 #pragma unroll
           for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int q = 0; q < kU; ++q)
-              if (sp + j < S && bq[q] >= 0 && bq[q] < p.batch) {
-                const float4* os = op + base[q] + static_cast<long>(sp + j) * dq * H;
-                x[j][q][0] = os[0];
-                x[j][q][1] = os[H];
-              }
+              if (sp + j < S && bq[q] >= 0 && bq[q] < p.batch)
+                x[j][q] = op[base[q] + static_cast<long>(sp + j) * d8 * H];
 #pragma unroll
           for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int q = 0; q < kU; ++q)
               if (sp + j < S && bq[q] >= 0 && bq[q] < p.batch) {
                 const float w = wts[bq[q] * S + sp + j];
-                const float4 x0 = x[j][q][0], x1 = x[j][q][1];
+                const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&x[j][q].x));
+                const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&x[j][q].y));
+                const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&x[j][q].z));
+                const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&x[j][q].w));
+                const float4 x0 = make_float4(f0.x, f0.y, f1.x, f1.y), x1 = make_float4(f2.x, f2.y, f3.x, f3.y);
                 float* a = acc[q];
                 a[0] += w * x0.x; a[1] += w * x0.y; a[2] += w * x0.z; a[3] += w * x0.w;
                 a[4] += w * x1.x; a[5] += w * x1.y; a[6] += w * x1.z; a[7] += w * x1.w;

@@ -2,6 +2,7 @@
 // kernel translation units.  Not part of the public interface (include/mla.h).
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -87,7 +88,9 @@ struct DecodeArgs {
   const float* cache_scale;   // [num_blocks, block_size] (fp8)
   const int32_t* block_table; // [B, max_blocks]
   const int32_t* seq_lens;    // [B]
-  float* o_part;              // [B, S, d_c/4, H, 4]
+  // split partials: bf16 activations: fp16 [B, S, d_c/8, H, 8]; fp32
+  // activations: fp32 [B, S, d_c/4, H, 4] (16 bytes per head and column group)
+  void* o_part;
   float* lse_part;            // [B, S, H]
   int* err;
   int32_t batch, num_heads, d_c, d_r, block_size, max_blocks, num_splits, num_blocks;
@@ -97,7 +100,7 @@ struct DecodeArgs {
 };
 
 struct CombineArgs {
-  const float* o_part;
+  const void* o_part;         // as DecodeArgs::o_part
   const float* lse_part;
   void* o_lat;                // [B, H, d_c] act dtype
   float* lse;                 // [B, H] or null
@@ -114,7 +117,7 @@ struct OutProjArgs {
   int32_t batch, num_heads, d_c, d_v, d_model;
   // merge fused into W_UV: o_lat (then an output) is built from the split-KV
   // partials; comb_splits = 0 turns this off
-  const float* comb_opart;   // [B, S, d_c/4, H, 4]
+  const __half* comb_opart;  // fp16 [B, S, d_c/8, H, 8]
   const float* comb_lse;     // [B, S, H]
   int32_t comb_splits;
   float* comb_lse_out;       // [B, H] or null

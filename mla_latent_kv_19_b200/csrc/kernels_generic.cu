@@ -7,6 +7,7 @@
 //
 // Method: DeepSeek V2 MLA page (snabindia.com), sections 2.1-2.3.
 #include <algorithm>
+#include <type_traits>
 
 #include "device_common.cuh"
 
@@ -377,8 +378,10 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(DecodeArgs 
   }
   __syncthreads();
   const long part = (static_cast<long>(b) * a.num_splits + split) * a.num_heads;
-  // o_part[b][s][c/4][h][c%4]
-  float* obase = a.o_part + (static_cast<long>(b) * a.num_splits + split) * a.d_c * a.num_heads;
+  // o_part[b][s][c/4][h][c%4] in fp32 (fp32 activations) or [c/8][h][c%8] in
+  // fp16 (bf16 activations)
+  const long obase = (static_cast<long>(b) * a.num_splits + split) * a.d_c * a.num_heads;
+  float big = 0.f;
 #pragma unroll
   for (int jc = 0; jc < kGenColsPerThread; ++jc) {
     const int c = tid + jc * kGenThreads;
@@ -387,11 +390,19 @@ __global__ void __launch_bounds__(kGenThreads) decode_generic_kernel(DecodeArgs 
       for (int g = 0; g < kGenHeads; ++g) {
         if (g < nh) {
           const float l = ps[g];
-          obase[((c >> 2) * a.num_heads + h0 + g) * 4 + (c & 3)] = l > 0.f ? acc[g][jc] / l : 0.f;
+          const float x = l > 0.f ? acc[g][jc] / l : 0.f;
+          if constexpr (std::is_same<T, float>::value) {
+            static_cast<float*>(a.o_part)[obase + ((c >> 2) * a.num_heads + h0 + g) * 4 + (c & 3)] = x;
+          } else {
+            big = fmaxf(big, fabsf(x));
+            static_cast<__half*>(a.o_part)[obase + ((c >> 3) * a.num_heads + h0 + g) * 8 + (c & 7)] =
+                __float2half_rn(x);
+          }
         }
       }
     }
   }
+  if (!(big <= 65504.f)) report_error(a.err, MLA_ERR_RANGE);
   if (tid < nh) {
     const float l = ps[tid];
     a.lse_part[part + h0 + tid] =
@@ -458,8 +469,10 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
     const float inv_z = z > 0.f ? 1.f / z : 0.f;
     if (blockIdx.y == 0 && a.lse != nullptr)
       a.lse[static_cast<long>(b) * H + h] = z > 0.f ? m + __logf(z) : -INFINITY;
-    const float4* op = reinterpret_cast<const float4*>(a.o_part) +
-                       (static_cast<long>(b) * S * a.d_c + c0) / 4 * H + h;
+    // o_part: fp32 [b][s][c/4][h][4] with fp32 activations, fp16 [b][s][c/8][h][8]
+    // with bf16 ones; a 4-column group c.. is then half (c/4) & 1 of 16 bytes
+    constexpr bool kF32 = std::is_same<T, float>::value;
+    const long obase = static_cast<long>(b) * S * a.d_c * H;
     float acc[kCols];
 #pragma unroll
     for (int c = 0; c < kCols; ++c) acc[c] = 0.f;
@@ -467,11 +480,21 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
 #pragma unroll 2
     for (int s = 0; s < S; ++s) {
       const float w = cw[s * H + h];
-      const float4* os = op + static_cast<long>(s) * (a.d_c / 4) * H;
+      const long sbase = obase + static_cast<long>(s) * a.d_c * H;
 #pragma unroll
       for (int g = 0; g < kCols / 4; ++g) {
         if (g < nq) {
-          const float4 v = os[g * H];
+          const int c = c0 + 4 * g;
+          float4 v;
+          if constexpr (kF32) {
+            v = reinterpret_cast<const float4*>(static_cast<const float*>(a.o_part) + sbase)[(c >> 2) * H + h];
+          } else {
+            const uint2 u = *reinterpret_cast<const uint2*>(static_cast<const __half*>(a.o_part) + sbase +
+                                                            ((c >> 3) * H + h) * 8 + (c & 7));
+            const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+            const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+            v = make_float4(lo.x, lo.y, hi.x, hi.y);
+          }
           acc[4 * g] += w * v.x;
           acc[4 * g + 1] += w * v.y;
           acc[4 * g + 2] += w * v.z;

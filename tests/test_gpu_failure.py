@@ -62,3 +62,32 @@ def test_out_of_range_page_in_decode_is_reported_not_read(name):
     r = oracle.step_outputs(wl, [0, 2], fp8_dequant=wl.cache_dtype == "fp8_e4m3")
     assert_close("o_lat", g["o_lat"][[0, 2]], r["o_lat"])
     assert np.all(np.isfinite(g["o_lat"][1]))
+
+
+def test_partial_beyond_fp16_range_is_reported():
+    """With bf16 activations the split partials are kept in fp16.  A latent
+    output beyond +-65504 (here: every cached row of one sequence set to 1e5,
+    so that o_lat is 1e5 whatever the softmax) records MLA_ERR_RANGE rather
+    than passing an infinity on; the other sequence and the next call are
+    unaffected."""
+    from mla_latent_kv_19_b200 import mla_last_device_error
+    from mla_latent_kv_19_b200.step import DecodeStep
+    wl = workloads.make("v2_b32_l2048", batch=2, context=300)
+    st = DecodeStep(wl, num_splits=2)
+    st.run()
+    assert mla_last_device_error(st.h) == 0
+    bt = st.block_table.cpu().numpy()
+    rows = [int(p) * 64 + j for p in bt[1, :(int(wl.seq_lens[1]) + 63) // 64] for j in range(64)]
+    saved = st.cache[rows].clone()
+    st.cache[rows] = 1e5
+    st.decode_partial()
+    st.decode_combine()
+    assert mla_last_device_error(st.h) == -9    # MLA_ERR_RANGE
+    st.cache[rows] = saved
+    st.decode_partial()
+    st.decode_combine()
+    assert mla_last_device_error(st.h) == 0
+    g = st.outputs()
+    st.close()
+    r = oracle.step_outputs(wl)
+    assert_close("o_lat", g["o_lat"], r["o_lat"])

@@ -219,10 +219,10 @@ def test_combine_against_oracle_merge():
     o[1, :, 5] = 0
     nbytes = mla_decode_workspace_bytes(h, B, S, 64 * S)
     ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
-    n_o = B * S * H * dc * 4
-    # workspace layout o_part[b][s][c/4][h][c%4]
-    packed = o.reshape(B, S, H, dc // 4, 4).transpose(0, 1, 3, 2, 4)
-    ws[:n_o].view(torch.float32).copy_(torch.from_numpy(np.ascontiguousarray(packed).reshape(-1)))
+    n_o = B * S * H * dc * 2
+    # workspace layout (bf16 activations): fp16 o_part[b][s][c/8][h][c%8]
+    packed = o.astype(np.float16).reshape(B, S, H, dc // 8, 8).transpose(0, 1, 3, 2, 4)
+    ws[:n_o].view(torch.float16).copy_(torch.from_numpy(np.ascontiguousarray(packed).reshape(-1)))
     off = (n_o + 255) // 256 * 256
     ws[off:off + B * S * H * 4].view(torch.float32).copy_(torch.from_numpy(lse.reshape(-1)))
     o_lat = torch.empty(B, H, dc, dtype=torch.bfloat16, device="cuda")
