@@ -285,9 +285,13 @@ __global__ void __launch_bounds__(256, 1)
     float* invz = wts + p.n * S;
     for (int b = ct; b < p.n; b += kCombThreads) {
       float mm = -INFINITY;
-      if (b < p.batch)
+      // (unrolled: eight loads in flight rather than one round trip per split)
+      if (b < p.batch) {
+#pragma unroll 8
         for (int sp = 0; sp < S; ++sp) mm = fmaxf(mm, p.comb_lse[(static_cast<long>(b) * S + sp) * H + h]);
+      }
       float z = 0.f;
+#pragma unroll 8
       for (int sp = 0; sp < S; ++sp) {
         const float w = (b >= p.batch || mm == -INFINITY) ? 0.f
                                                            : __expf(p.comb_lse[(static_cast<long>(b) * S + sp) * H + h] - mm);
