@@ -41,6 +41,7 @@ def test_status_strings():
     assert m.mla_status_string(0) == "MLA_OK"
     assert m.mla_status_string(-6) == "MLA_ERR_BAD_INDEX"
     assert m.mla_status_string(-7) == "MLA_ERR_TIMEOUT"
+    assert m.mla_status_string(-9) == "MLA_ERR_RANGE"
     assert m.mla_status_string(12345) == "MLA_ERR_UNKNOWN"
 
 
@@ -89,6 +90,11 @@ def test_null_arguments():
     assert m.lib.mla_out_proj(null, None, None, None, 1, None, 0, None, None, None) == -1
     assert m.lib.mla_last_device_error(null, None) == -1
     assert m.lib.mla_set_wait_limit(null, 5) == -1
+    assert m.lib.mla_set_launch_overlap(null, 1) == -1
+    assert m.lib.mla_set_w_o_layout(null, 1) == -1
+    assert m.lib.mla_pack_w_o(null, None, None, None) == -1
+    assert m.lib.mla_combine_out_proj(null, 1, 64, 1, None, 0, None, None, None, 0, None, None, None, None,
+                                      None) == -1
 
 
 def test_create_without_device_reports_cuda_error():
