@@ -58,7 +58,7 @@ extern "C" {
 typedef enum {
   MLA_OK = 0,
   MLA_ERR_INVALID_ARG = -1,  /* null pointer, bad size or bad config value        */
-  MLA_ERR_UNSUPPORTED = -2,  /* dims/dtypes this build has no kernel for            */
+  MLA_ERR_UNSUPPORTED = -2,  /* dims/dtypes the library has no kernel for          */
   MLA_ERR_ALIGNMENT = -3,    /* a pointer is not 16-byte aligned                   */
   MLA_ERR_WORKSPACE = -4,    /* workspace null or smaller than the query call says */
   MLA_ERR_LAUNCH = -5,       /* a kernel launch failed (cudaGetLastError)          */

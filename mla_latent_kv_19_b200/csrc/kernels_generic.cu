@@ -88,9 +88,9 @@ __device__ void write_row_warp_fp8(const AppendArgs& a, const float* stage, long
   if (lane == 0) a.cache_scale[slot] = amax / 448.f;
 }
 
-// One warp per token.  Round 1 loads the token's sequence, position and values
-// together; round 2 the page-table entry and the RoPE factors, which depend on
-// them; then the row is rotated, converted and written.  An out-of-range
+// One warp per token.  The first memory round trip loads the token's sequence,
+// position and values together; the second the page-table entry and the RoPE
+// factors, which depend on them; then the row is rotated, converted and written.  An out-of-range
 // sequence, position or page is reported and the token skipped.
 template <typename T, typename CT, bool kFp8, bool kProject>
 __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(AppendArgs a) {
